@@ -1,0 +1,349 @@
+#!/usr/bin/env python
+"""Benchmark of the any4 linear layer on B200.
+
+Workload: the linear stack of Llama-3-8B (32 decoder layers x {q 4096x4096,
+k 1024x4096, v 1024x4096, o 4096x4096, gate 14336x4096, up 14336x4096,
+down 4096x14336}), any4 with group 128, run back to back at M = 1 and then at
+M = 16. One step = both passes = 448 any4_linear calls. Weights are synthetic
+any4 tensors (one drawn set per distinct shape, packed once, copied to 32
+distinct device buffers: 3.76 GB, far above the 126 MB L2, so every call
+streams its weights from HBM). Activations are per call.
+
+Output: one JSON line (rank 0). ``value`` is the aggregate algorithmic HBM
+throughput in GB/s (packed indices, LUTs, alpha/beta, x and y bytes of every
+call of every rank / the max over ranks of the step time).
+
+``--impl reference`` times the CPU oracle on the same workload and metric,
+each step a bounded sample of the stack.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+GROUP = 128
+LAYERS = 32
+MS = (1, 16)
+FALLBACK_HBM_GBS = 6650.0
+
+
+def algorithmic_bytes(m: int, n: int, k: int, g: int) -> int:
+    return n * k // 2 + n * (k // g) * 4 + n * 32 + m * k * 2 + m * n * 2
+
+
+def stack_calls():
+    """(m, layer, shape) for one step, in execution order."""
+    return [(m, layer, sh) for m in MS for layer in range(LAYERS) for sh in synth.LLAMA3_8B_LAYER]
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], 0
+        self._stop = threading.Event()
+        self.ok = True
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.ok = False
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml_unavailable"],
+                    "samples": 0}
+        names = [v for b, v in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+def cpu_baseline(budget_s: float, calls=None):
+    """Time the oracle on the stack's calls, in order, for about ``budget_s``."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        blas = 1
+    calls = calls or stack_calls()
+    cache, xs = {}, {}
+    done_bytes, t_total, count = 0, 0.0, 0
+    for (m, layer, sh) in calls:
+        key = (sh.n, sh.k)
+        if key not in cache:
+            idx, lut, a, b = synth.random_any4(sh.n, sh.k, GROUP, 0, layer=sh.name)
+            cache[key] = oracle.Any4Tensors(idx, lut, a, b, GROUP)
+        s = synth.channel_scale(sh.k, 0, layer=sh.name)
+        x = synth.activations_bf16(m, s, layer, layer=sh.name)
+        t0 = time.perf_counter()
+        oracle.linear(x, cache[key])
+        t_total += time.perf_counter() - t0
+        done_bytes += algorithmic_bytes(m, sh.n, sh.k, GROUP)
+        count += 1
+        if t_total >= budget_s:
+            break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(max(1, blas)),
+            "kind": "oracle",
+            "sample": f"first {count} of {len(calls)} calls of one step (M=1 pass first), "
+                      f"{t_total:.1f} s: fp64 bit-exact dequant (single-threaded numpy) + "
+                      f"fp64 matmul ({blas} BLAS threads)"}
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    calls = stack_calls()
+    step_bytes_full = sum(algorithmic_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
+    per_step_budget = max(0.5, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(per_step_budget, calls)
+        if i >= args.warmup:
+            vals.append(r)
+    value = float(np.mean([v["value"] for v in vals]))
+    ms_per_step = step_bytes_full / (value * 1e9) * 1e3
+    line = {"impl": "reference", "metric": "any4_linear achieved HBM GB/s (algorithmic bytes)",
+            "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS, "ms": list(MS),
+                       "group": GROUP, "calls_per_step": len(calls)},
+            "cpu_baseline": {**vals[-1], "value": value},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+
+    import learned_bit_lut_b200 as a4
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+
+    calls = stack_calls()
+    # packed weights: one drawn set per distinct shape, copied to 32 layers
+    packed = {}
+    for sh in synth.LLAMA3_8B_LAYER:
+        idx, lut, al, be = synth.random_any4(sh.n, sh.k, GROUP, 0, layer=sh.name)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+        base = a4.any4_pack(t(idx), t(lut), t(al), t(be), GROUP)
+        for layer in range(LAYERS):
+            packed[(layer, sh.name)] = base if layer == 0 else base.clone()
+    del base
+    # activations and outputs per call (one flat device buffer each)
+    xoff, yoff, xo, yo = [], [], 0, 0
+    for (m, layer, sh) in calls:
+        xoff.append(xo); yoff.append(yo)
+        xo += m * sh.k
+        yo += m * sh.n
+    x_host = np.empty(xo, dtype=np.uint16)
+    for i, (m, layer, sh) in enumerate(calls):
+        s = synth.channel_scale(sh.k, 0, layer=sh.name)
+        x_host[xoff[i]:xoff[i] + m * sh.k] = synth.activations_bf16(m, s, 1000 + layer, layer=sh.name).ravel()
+    x_dev = torch.from_numpy(x_host.view(np.int16)).to(dev).view(torch.bfloat16)
+    y_dev = torch.empty(yo, dtype=torch.bfloat16, device=dev)
+    ws_need = max(a4.any4_linear_workspace_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
+    ws = torch.zeros(ws_need, dtype=torch.uint8, device=dev)
+
+    def issue(sel):
+        for i in sel:
+            m, layer, sh = calls[i]
+            a4.any4_linear(x_dev[xoff[i]:xoff[i] + m * sh.k].view(m, sh.k),
+                           packed[(layer, sh.name)], sh.n, sh.k, GROUP,
+                           out=y_dev[yoff[i]:yoff[i] + m * sh.n].view(m, sh.n), workspace=ws)
+
+    sel = {mm: [i for i, c in enumerate(calls) if c[0] == mm] for mm in MS}
+    graphs = {}
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        issue(range(len(calls)))          # eager warm-up before capture
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    for mm in MS:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            issue(sel[mm])
+        graphs[mm] = g
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, steps):
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    def step():
+        for mm in MS:
+            graphs[mm].replay()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        ms_total = timed(step, args.steps)
+    ms_step = ms_total / args.steps
+    per_m = {}
+    for mm in MS:
+        for _ in range(2):
+            graphs[mm].replay()
+        ms_m = timed(graphs[mm].replay, args.steps) / args.steps
+        b = sum(algorithmic_bytes(mm, sh.n, sh.k, GROUP) for m, _, sh in calls if m == mm)
+        per_m[str(mm)] = {"us_per_call": ms_m * 1e3 / len(sel[mm]), "GB/s": b / (ms_m * 1e6)}
+
+    step_bytes = sum(algorithmic_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
+    value = step_bytes * world / (ms_step * 1e6)
+    peak, peak_kind = read_peaks()
+    achieved = step_bytes / (ms_step * 1e6)
+
+    # end to end through the Python API: pinned host x in, y out, every step
+    e2e = None
+    if not args.no_e2e:
+        x_pin = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+        y_pin = torch.empty(yo, dtype=torch.int16).pin_memory()
+        x_in = torch.empty_like(x_dev)
+        y_out = torch.empty_like(y_dev)
+
+        def e2e_step():
+            x_in.view(torch.int16).copy_(x_pin, non_blocking=True)
+            for i, (m, layer, sh) in enumerate(calls):
+                a4.any4_linear(x_in[xoff[i]:xoff[i] + m * sh.k].view(m, sh.k),
+                               packed[(layer, sh.name)], sh.n, sh.k, GROUP,
+                               out=y_out[yoff[i]:yoff[i] + m * sh.n].view(m, sh.n), workspace=ws)
+            y_pin.copy_(y_out.view(torch.int16), non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        e2e_steps = max(3, min(args.steps, 20))
+        ms_e2e = timed(e2e_step, e2e_steps) / e2e_steps
+        e2e = {"value": step_bytes * world / (ms_e2e * 1e6), "unit": "GB/s",
+               "h2d_bytes_per_step": int(x_host.nbytes), "d2h_bytes_per_step": int(yo * 2),
+               "ms_per_step": ms_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": "any4_linear achieved HBM GB/s (algorithmic bytes)",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS,
+                       "linears_per_layer": len(synth.LLAMA3_8B_LAYER), "ms": list(MS),
+                       "group": GROUP, "calls_per_step": len(calls),
+                       "l2": "inputs larger than L2: 3.76 GB of distinct packed weights per step",
+                       "parallelism": f"replicas x{world}"},
+            "us_per_call": ms_step * 1e3 / len(calls),
+            "by_m": per_m,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs", "kernel": "linear_kernel"},
+            "gpu_launches": len(calls) * args.steps,
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    for g in graphs.values():
+        del g
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

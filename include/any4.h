@@ -1,0 +1,140 @@
+/*
+ * any4.h - C ABI of the any4 mixed-precision linear layer for NVIDIA B200 (sm_100a).
+ *
+ * any4 stores every weight of a linear layer W (N x K, one row per output
+ * channel) as a 4-bit index into a per-row table (LUT) of 16 bf16 values; each
+ * row is split into contiguous groups of G columns with a bf16 scale alpha and
+ * offset beta per group. The dequantized weight is
+ *
+ *     w_hat[n][k] = fma(alpha[n][k/G], LUT[n][idx[n][k]], beta[n][k/G])
+ *
+ * Sources: the any4 explainer (10100.com, article 149119421), section 2 (per-row
+ * 16-entry FP16/BF16 table, 4-bit index per weight, table read at inference),
+ * section 2.1 (per-group scale and offset), section 3 (tinygemm: table held in
+ * registers, weights pre-arranged in the compute format, batch 1-16 decode);
+ * "any4: Learned 4-bit Numeric Representation for LLMs" (arXiv 2507.04610,
+ * abstract).
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates, frees or keeps a reference to caller memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronize the device.
+ *  - bf16 values are passed as their 16-bit patterns (uint16_t).
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns a negative any4_status and launches nothing.
+ *  - A failed kernel launch returns ANY4_ECUDA; the CUDA error code is kept
+ *    per thread and returned by any4_last_cuda_error().
+ *  - Accepted shapes: N > 0 and N % 16 == 0; K > 0 and K % 64 == 0;
+ *    G in {64, 128, 256, 512, 1024} and K % G == 0; 1 <= M <= 16.
+ *    Anything else returns ANY4_ESHAPE.
+ */
+#ifndef ANY4_H
+#define ANY4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of the shared library are exported explicitly (it is built with
+ * hidden default visibility). */
+#if defined(__GNUC__)
+#define ANY4_API __attribute__((visibility("default")))
+#else
+#define ANY4_API
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* any4_stream_t;
+
+typedef enum {
+    ANY4_OK = 0,
+    ANY4_EINVAL = -1,      /* null pointer or a negative / zero size           */
+    ANY4_EALIGN = -2,      /* a pointer misses its required alignment          */
+    ANY4_ESHAPE = -3,      /* M, N, K or G outside the accepted set            */
+    ANY4_EWORKSPACE = -4,  /* packed buffer or workspace smaller than required */
+    ANY4_ECUDA = -5        /* a CUDA runtime call or kernel launch failed      */
+} any4_status;
+
+/*
+ * Size in bytes of the device-layout buffer any4_pack writes for an N x K
+ * weight with group size G; 0 if the shape is not accepted. The size is
+ * N*K/2 (indices) + 32*N (LUT) + 4*N*(K/G) (alpha and beta), each section
+ * padded to 256 bytes. At K = 4096 the LUT adds 16*16/4096 = 0.0625 bit per
+ * weight (explainer section 2.3).
+ */
+ANY4_API size_t any4_packed_bytes(int n, int k, int group);
+
+/*
+ * any4_pack - reorder canonical any4 tensors into the device layout
+ * (explainer section 3: weights pre-arranged in the hardware compute format).
+ *
+ *   idx_nib  [N][K/2] uint8: byte j of row n holds the index of column 2j in
+ *            its low nibble and of column 2j+1 in its high nibble.
+ *   lut      [N][16]  bf16 table of each row (section 2).
+ *   alpha    [N][K/G] bf16 group scales; beta [N][K/G] bf16 group offsets
+ *            (section 2.1).
+ *   packed   output, packed_bytes >= any4_packed_bytes(n, k, group); 16-byte
+ *            aligned. The layout is opaque and immutable once written; it may
+ *            be read by any number of calls and streams.
+ * Inputs need no particular alignment. Returns ANY4_OK or an error status.
+ */
+ANY4_API int any4_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint16_t* alpha,
+              const uint16_t* beta, int n, int k, int group, void* packed,
+              size_t packed_bytes, any4_stream_t stream);
+
+/*
+ * any4_dequant - debug call: write the dequantized weight matrix.
+ *   w  output [N][K] bf16, row-major, 4-byte aligned.
+ * w_hat[n][k] is alpha*LUT[idx]+beta evaluated as one fp32 fused
+ * multiply-add rounded to nearest-even, then rounded to bf16 nearest-even
+ * (subnormals kept). Bit-exact by construction.
+ */
+ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t* w,
+                 any4_stream_t stream);
+
+/*
+ * Bytes of workspace any4_linear needs for this shape on the CURRENT device
+ * (the launch is sized by the device's SM count); 0 if the shape is not
+ * accepted. The workspace holds fp32 partial sums of output tiles split along
+ * K and one 32-bit arrival counter per 16-row tile.
+ */
+ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
+
+/*
+ * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
+ *
+ *   x          [M][K] bf16 activations, row-major, 16-byte aligned.
+ *   packed     the any4_pack output for W (N x K, group G).
+ *   y          [M][N] bf16 output, row-major, 4-byte aligned.
+ *   workspace  >= any4_linear_workspace_bytes(m, n, k, group) bytes, 16-byte
+ *              aligned, owned by the caller. It MUST be zero-filled before its
+ *              first use: it starts with the per-tile arrival counters, and
+ *              every call that runs to completion sets them back to zero (the
+ *              partial-sum area behind them needs no initialization). After a
+ *              failed launch, zero-fill it again. Calls that may overlap on
+ *              the device need separate workspaces.
+ *
+ * Each weight is dequantized as w_hat = fma(alpha, LUT[idx], beta) in bf16
+ * (fma.rn.bf16x2: the exact value rounded once to bf16) and contracted on the
+ * tensor cores with fp32 accumulation; the fp32 result is rounded to bf16
+ * nearest-even. Tiles split along K are reduced in a fixed order, so the
+ * result is deterministic.
+ */
+ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
+                uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+ANY4_API const char* any4_strerror(int status);
+
+/* The cudaError_t value of the last ANY4_ECUDA returned on this host thread. */
+ANY4_API int any4_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ANY4_H */

@@ -1,0 +1,149 @@
+"""ctypes binding of libany4.so (include/any4.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, and their device pointers plus the current CUDA stream are passed
+to the C ABI. Every step of the computation runs in the library's kernels;
+there is no fallback path. Importing this module fails loudly when the
+library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libany4.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m learned_bit_lut_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_c_size = ctypes.c_size_t
+_c_int = ctypes.c_int
+_p = ctypes.c_void_p
+
+lib.any4_packed_bytes.argtypes = [_c_int, _c_int, _c_int]
+lib.any4_packed_bytes.restype = _c_size
+lib.any4_pack.argtypes = [_p, _p, _p, _p, _c_int, _c_int, _c_int, _p, _c_size, _p]
+lib.any4_pack.restype = _c_int
+lib.any4_dequant.argtypes = [_p, _c_int, _c_int, _c_int, _p, _p]
+lib.any4_dequant.restype = _c_int
+lib.any4_linear_workspace_bytes.argtypes = [_c_int, _c_int, _c_int, _c_int]
+lib.any4_linear_workspace_bytes.restype = _c_size
+lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
+lib.any4_linear.restype = _c_int
+lib.any4_strerror.argtypes = [_c_int]
+lib.any4_strerror.restype = ctypes.c_char_p
+lib.any4_last_cuda_error.argtypes = []
+lib.any4_last_cuda_error.restype = _c_int
+
+EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
+            "any4_linear", "any4_strerror", "any4_last_cuda_error")
+
+ANY4_OK, ANY4_EINVAL, ANY4_EALIGN, ANY4_ESHAPE, ANY4_EWORKSPACE, ANY4_ECUDA = 0, -1, -2, -3, -4, -5
+
+
+class Any4Error(RuntimeError):
+    def __init__(self, status: int):
+        msg = lib.any4_strerror(status).decode()
+        if status == ANY4_ECUDA:
+            msg += f" (cudaError {lib.any4_last_cuda_error()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status != ANY4_OK:
+        raise Any4Error(status)
+
+
+def _dev(t: torch.Tensor, name: str, itemsize: int, shape=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.element_size() != itemsize:
+        raise ValueError(f"{name} must have {itemsize}-byte elements, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def any4_packed_bytes(n: int, k: int, group: int) -> int:
+    return lib.any4_packed_bytes(n, k, group)
+
+
+def any4_linear_workspace_bytes(m: int, n: int, k: int, group: int) -> int:
+    return lib.any4_linear_workspace_bytes(m, n, k, group)
+
+
+def any4_pack(idx_nib: torch.Tensor, lut: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+              group: int, packed: torch.Tensor | None = None) -> torch.Tensor:
+    """Canonical any4 tensors -> device-layout buffer (uint8 tensor)."""
+    n, k2 = idx_nib.shape
+    k = 2 * k2
+    size = any4_packed_bytes(n, k, group)
+    if size == 0:
+        raise Any4Error(ANY4_ESHAPE)
+    dev = idx_nib.device
+    if packed is None:
+        packed = torch.empty(size, dtype=torch.uint8, device=dev)
+    _check(lib.any4_pack(_dev(idx_nib, "idx_nib", 1, (n, k2)), _dev(lut, "lut", 2, (n, 16)),
+                         _dev(alpha, "alpha", 2, (n, k // group)),
+                         _dev(beta, "beta", 2, (n, k // group)), n, k, group,
+                         _dev(packed, "packed", 1), packed.numel(), _stream(dev)))
+    return packed
+
+
+def any4_dequant(packed: torch.Tensor, n: int, k: int, group: int,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """Device-layout buffer -> dequantized W (N x K, bf16)."""
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=packed.device)
+    _check(lib.any4_dequant(_dev(packed, "packed", 1), n, k, group, _dev(out, "out", 2, (n, k)),
+                            _stream(packed.device)))
+    return out
+
+
+_WORKSPACES: dict = {}
+
+
+def workspace_for(m: int, n: int, k: int, group: int, device: torch.device) -> torch.Tensor:
+    """A zero-initialised workspace for this stream, grown on demand and reused
+    by later calls on the same stream (calls on one stream never overlap)."""
+    need = any4_linear_workspace_bytes(m, n, k, group)
+    if need == 0:
+        raise Any4Error(ANY4_ESHAPE)
+    key = (device.index if device.index is not None else torch.cuda.current_device(),
+           _stream(device))
+    ws = _WORKSPACES.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
+
+
+def any4_linear(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: int,
+                out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y = x . W_hat^T for bf16 x (M x K, M <= 16) -> y (M x N, bf16)."""
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(m, n, k, group, x.device)
+    _check(lib.any4_linear(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
+                           _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
+                           workspace.numel(), _stream(x.device)))
+    return out
+
+
+def any4_strerror(status: int) -> str:
+    return lib.any4_strerror(status).decode()

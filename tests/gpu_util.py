@@ -1,0 +1,101 @@
+"""Helpers shared by the GPU parity tests: canonical any4 tensors from the
+oracle (or drawn directly for full-size shapes), device copies, and the
+comparison rules."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+
+# Acceptance bar of the linear layer: per token row m,
+#   max_n |y - y_ref| <= REL_TOL * max_n |y_ref|.
+REL_TOL = 2e-2
+
+
+def require_gpu():
+    assert torch.cuda.is_available(), "these tests need a CUDA GPU"
+    return torch.device("cuda:0")
+
+
+def to_dev(a: np.ndarray, device="cuda:0") -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device)
+    return torch.from_numpy(a).to(device)
+
+
+def bf16_dev(bits: np.ndarray, device="cuda:0") -> torch.Tensor:
+    return to_dev(bits, device).view(torch.bfloat16)
+
+
+def bits_host(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def calib(k: int, seed: int, layer: str, sigma: float = 0.5):
+    s = synth.channel_scale(k, seed, sigma=sigma, layer=layer)
+    ex = oracle.calibrate(synth.calibration_acts(512, s, seed, layer=layer))
+    return s, ex
+
+
+@functools.lru_cache(maxsize=None)
+def quantized(n: int, k: int, g: int, seed: int = 0, layer: str = "w", kind: str = "normal",
+              sigma: float = 0.5, iters: int = 10):
+    """Oracle-quantized weight (all rows) and its activation scale."""
+    w = synth.weights_bf16(n, k, seed, kind=kind, layer=layer)
+    s, ex = calib(k, seed, layer, sigma)
+    return oracle.quantize(w, ex, g=g, iters=iters), s
+
+
+@functools.lru_cache(maxsize=None)
+def mixed(n: int, k: int, g: int, rows: tuple, seed: int = 0, layer: str = "w",
+          kind: str = "normal", sigma: float = 0.5):
+    """Full-size any4 tensors: directly drawn rows everywhere, oracle-quantized
+    rows (k-means on synthetic weights of the workload's distribution) at
+    ``rows``. Returns (tensors, activation scale)."""
+    idx, lut, a, b = synth.random_any4(n, k, g, seed, layer=layer)
+    w = synth.weights_bf16(len(rows), k, seed, kind=kind, layer=layer + "/rows")
+    s, ex = calib(k, seed, layer, sigma)
+    q = oracle.quantize(w, ex, g=g, iters=10)
+    r = np.asarray(rows)
+    idx[r], lut[r], a[r], b[r] = q.idx_nib, q.lut, q.alpha, q.beta
+    return oracle.Any4Tensors(idx, lut, a, b, g), s
+
+
+def sample_rows(n: int, count: int = 48, seed: int = 0) -> tuple:
+    """Rows of the first and last tiles plus spread random rows."""
+    g = np.random.default_rng(seed)
+    pick = set(range(min(16, n))) | set(range(max(0, n - 16), n))
+    pick |= set(g.choice(n, size=min(n, count), replace=False).tolist())
+    return tuple(sorted(pick))
+
+
+def pack_dev(q: oracle.Any4Tensors, device="cuda:0"):
+    import learned_bit_lut_b200 as a4
+    return a4.any4_pack(to_dev(q.idx_nib, device), to_dev(q.lut, device), to_dev(q.alpha, device),
+                        to_dev(q.beta, device), q.group)
+
+
+def check_linear(y_gpu: torch.Tensor, x_bits: np.ndarray, q: oracle.Any4Tensors, rows=None):
+    """Compare y (M x N, bf16 on the GPU) with the oracle on ``rows`` (all if None).
+
+    Two bars: the acceptance bar (REL_TOL of each token row's max |y_ref|) and
+    a tight elementwise bar (half a bf16 ulp of the output plus fp32
+    accumulation error), since the kernel contracts the same bf16 weights.
+    """
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    ref = oracle.linear_rows(x_bits, q, rows)
+    if rows is not None:
+        y = y[:, np.asarray(rows)]
+    scale = np.max(np.abs(ref), axis=1, keepdims=True)
+    err = np.abs(y - ref)
+    worst = np.max(err / np.maximum(scale, 1e-30), axis=1)
+    assert np.all(worst <= REL_TOL), f"relative error per token {worst}"
+    tight = np.abs(ref) * 2.0 ** -8 + 1e-4 * scale
+    bad = np.argwhere(err > tight)
+    assert bad.size == 0, f"{len(bad)} elements off, first {bad[:5].tolist()}"
+    return float(worst.max())

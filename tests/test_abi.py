@@ -1,0 +1,72 @@
+"""C ABI: the library loads, exports what include/any4.h declares, and rejects
+invalid calls on the host before any launch (CPU only, no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import learned_bit_lut_b200 as a4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "any4.h")).read()
+    return sorted(set(re.findall(r"ANY4_API\s+[\w\s\*]*?\b(any4_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = _declared()
+    assert names == sorted(a4.EXPORTED)
+    for n in names:
+        assert hasattr(a4.lib, n), n
+        assert ctypes.cast(getattr(a4.lib, n), ctypes.c_void_p).value
+
+
+def test_packed_bytes_accounting():
+    n, k, g = 4096, 4096, 128
+    total = a4.any4_packed_bytes(n, k, g)
+    idx, lut, ab = n * k // 2, 32 * n, 4 * n * (k // g)
+    assert total == idx + lut + ab            # all sections already 256-byte multiples here
+    assert lut * 8 / (n * k) == 0.0625        # explainer section 2.3
+    # padding: each section rounded up to 256 bytes
+    assert a4.any4_packed_bytes(16, 64, 64) == 512 + 512 + 256
+
+
+@pytest.mark.parametrize("n,k,g", [(0, 64, 64), (15, 64, 64), (16, 63, 64), (16, 64, 32),
+                                   (16, 192, 128), (16, 64, 96), (-16, 64, 64)])
+def test_bad_shapes(n, k, g):
+    assert a4.any4_packed_bytes(n, k, g) == 0
+    assert a4.any4_linear_workspace_bytes(1, n, k, g) == 0
+    p = ctypes.c_void_p(256)
+    assert a4.lib.any4_pack(p, p, p, p, n, k, g, p, 1 << 30, None) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_dequant(p, n, k, g, p, None) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear(p, p, 1, n, k, g, p, p, 1 << 30, None) == a4.ANY4_ESHAPE
+
+
+@pytest.mark.parametrize("m", [0, 17, -1])
+def test_bad_m(m):
+    p = ctypes.c_void_p(256)
+    assert a4.any4_linear_workspace_bytes(m, 64, 64, 64) == 0
+    assert a4.lib.any4_linear(p, p, m, 64, 64, 64, p, p, 1 << 30, None) == a4.ANY4_ESHAPE
+
+
+def test_null_and_misaligned_pointers():
+    p, z = ctypes.c_void_p(256), ctypes.c_void_p(0)
+    odd = ctypes.c_void_p(258)
+    assert a4.lib.any4_pack(z, p, p, p, 16, 64, 64, p, 4096, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_pack(p, p, p, p, 16, 64, 64, z, 4096, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_pack(p, p, p, p, 16, 64, 64, odd, 4096, None) == a4.ANY4_EALIGN
+    assert a4.lib.any4_pack(p, p, p, p, 16, 64, 64, p, 100, None) == a4.ANY4_EWORKSPACE
+    assert a4.lib.any4_dequant(z, 16, 64, 64, p, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_dequant(p, 16, 64, 64, ctypes.c_void_p(257), None) == a4.ANY4_EALIGN
+    assert a4.lib.any4_linear(z, p, 1, 16, 64, 64, p, p, 1 << 20, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_linear(odd, p, 1, 16, 64, 64, p, p, 1 << 20, None) == a4.ANY4_EALIGN
+    assert a4.lib.any4_linear(p, p, 1, 16, 64, 64, p, odd, 1 << 20, None) == a4.ANY4_EALIGN
+
+
+def test_strerror_covers_all_codes():
+    for code in (0, -1, -2, -3, -4, -5):
+        assert a4.any4_strerror(code).startswith("ANY4_")
+    assert "unknown" in a4.any4_strerror(7)

@@ -1,6 +1,7 @@
 """Build libany4.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m learned_bit_lut_b200.build [--force]``. The library is
+Usage: ``python learned_bit_lut_b200/build.py [--force]`` (run by path: importing
+the package loads the library). The library is
 rebuilt when a source or header is newer than it.
 """
 from __future__ import annotations

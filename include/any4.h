@@ -127,6 +127,29 @@ ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);
 
+/*
+ * any4_linear_noalloc - any4_linear for callers that cannot allocate device
+ * memory. The source pages have no counterpart of this call; it exists for
+ * callers such as operators running inside a serving runtime that owns all
+ * device memory and passes a kernel only its inputs and outputs, and
+ * latency-critical loops that must not call cudaMalloc because it can
+ * synchronize the device.
+ *
+ * Same arguments, result and rounding as any4_linear, minus the workspace:
+ * the partial sums and counters live in a fixed 8 MiB array of device memory
+ * that this library reserves on every GPU that loads it, until the process
+ * exits. A shape whose launch needs more than that returns ANY4_EWORKSPACE
+ * (on a 148-SM B200 all accepted shapes fit). The call allocates and frees
+ * nothing. The first call on a device looks up the array's address with that
+ * device current, so make it before any stream capture on that device. All
+ * calls on a device share the array: each call clears the counters it uses
+ * on `stream` before its kernel, and calls that can run at the same time on
+ * the GPU race and must be ordered by the caller. On ANY4_ECUDA the CUDA
+ * error code is not recorded for any4_last_cuda_error().
+ */
+ANY4_API int any4_linear_noalloc(const uint16_t* x, const void* packed, int m, int n, int k,
+                                 int group, uint16_t* y, any4_stream_t stream);
+
 /* Static description of a status code (never NULL). */
 ANY4_API const char* any4_strerror(int status);
 

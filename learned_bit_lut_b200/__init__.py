@@ -6,11 +6,11 @@ CUDA library does all the work; PyTorch only provides device memory and
 streams.
 """
 from ._lib import (ANY4_EALIGN, ANY4_ECUDA, ANY4_EINVAL, ANY4_ESHAPE, ANY4_EWORKSPACE, ANY4_OK,
-                   EXPORTED, LIB_PATH, Any4Error, any4_dequant, any4_linear,
+                   EXPORTED, LIB_PATH, Any4Error, any4_dequant, any4_linear, any4_linear_noalloc,
                    any4_linear_workspace_bytes, any4_pack, any4_packed_bytes, any4_strerror, lib,
                    workspace_for)
 
-__all__ = ["any4_pack", "any4_dequant", "any4_linear", "any4_packed_bytes",
+__all__ = ["any4_pack", "any4_dequant", "any4_linear", "any4_linear_noalloc", "any4_packed_bytes",
            "any4_linear_workspace_bytes", "any4_strerror", "Any4Error", "workspace_for", "lib",
            "LIB_PATH", "EXPORTED", "ANY4_OK", "ANY4_EINVAL", "ANY4_EALIGN", "ANY4_ESHAPE",
            "ANY4_EWORKSPACE", "ANY4_ECUDA"]

@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libany4.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m learned_bit_lut_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python learned_bit_lut_b200/build.py`")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -35,13 +35,15 @@ lib.any4_linear_workspace_bytes.argtypes = [_c_int, _c_int, _c_int, _c_int]
 lib.any4_linear_workspace_bytes.restype = _c_size
 lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
 lib.any4_linear.restype = _c_int
+lib.any4_linear_noalloc.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p]
+lib.any4_linear_noalloc.restype = _c_int
 lib.any4_strerror.argtypes = [_c_int]
 lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
-            "any4_linear", "any4_strerror", "any4_last_cuda_error")
+            "any4_linear", "any4_linear_noalloc", "any4_strerror", "any4_last_cuda_error")
 
 ANY4_OK, ANY4_EINVAL, ANY4_EALIGN, ANY4_ESHAPE, ANY4_EWORKSPACE, ANY4_ECUDA = 0, -1, -2, -3, -4, -5
 
@@ -142,6 +144,21 @@ def any4_linear(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: in
     _check(lib.any4_linear(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
                            _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
                            workspace.numel(), _stream(x.device)))
+    return out
+
+
+def any4_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: int,
+                        out: torch.Tensor | None = None) -> torch.Tensor:
+    """any4_linear without a workspace, for callers that cannot allocate device
+    memory (e.g. an operator inside a runtime that owns all device memory): the
+    library's own fixed scratch array is used instead. Calls that may overlap
+    on the GPU must be ordered by the caller, since they share that array.
+    ``out`` may be passed to avoid the one allocation this Python helper makes."""
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    _check(lib.any4_linear_noalloc(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k,
+                                   group, _dev(out, "out", 2, (m, n)), _stream(x.device)))
     return out
 
 

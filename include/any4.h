@@ -61,8 +61,9 @@ typedef enum {
 
 /*
  * Size in bytes of the device-layout buffer any4_pack writes for an N x K
- * weight with group size G; 0 if the shape is not accepted. The size is
- * N*K/2 (indices) + 32*N (LUT) + 4*N*(K/G) (alpha and beta), each section
+ * weight with group size G; 0 if the shape is not accepted. With Np = N
+ * rounded up to a multiple of 128 (the padding rows are zeros), the size is
+ * Np*K/2 (indices) + 32*Np (LUT) + 4*Np*(K/G) (alpha and beta), each section
  * padded to 256 bytes. At K = 4096 the LUT adds 16*16/4096 = 0.0625 bit per
  * weight (explainer section 2.3).
  */
@@ -99,8 +100,9 @@ ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t*
 /*
  * Bytes of workspace any4_linear needs for this shape on the CURRENT device
  * (the launch is sized by the device's SM count); 0 if the shape is not
- * accepted. The workspace holds fp32 partial sums of output tiles split along
- * K and one 32-bit arrival counter per 16-row tile.
+ * accepted. The workspace holds a fixed header of 8192 arrival counters (one
+ * per possible 128-row tile) and one error word, then the fp32 partial sums
+ * of output tiles split along K between thread blocks.
  */
 ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 
@@ -120,9 +122,11 @@ ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
  *
  * Each weight is dequantized as w_hat = fma(alpha, LUT[idx], beta) in bf16
  * (fma.rn.bf16x2: the exact value rounded once to bf16) and contracted on the
- * tensor cores with fp32 accumulation; the fp32 result is rounded to bf16
- * nearest-even. Tiles split along K are reduced in a fixed order, so the
- * result is deterministic.
+ * tensor cores (tcgen05) with fp32 accumulation; the fp32 result is rounded
+ * to bf16 nearest-even. Tiles split along K are reduced in a fixed order, so
+ * the result is deterministic. If an internal pipeline wait ever times out
+ * (about 2 s) the kernel stops, leaves y incomplete and sets a nonzero error
+ * word in the workspace header (byte offset 32768).
  */
 ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);

@@ -17,22 +17,21 @@ cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint1
 cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream);
 
+// The workspace of any4_linear starts with one arrival counter per possible
+// 128-row tile, so the counters of every shape live in the same zero-filled
+// header whatever the shape of earlier calls; then one error word; then the
+// fp32 partial tiles.
+constexpr int kMaxTiles = kMaxRows / kTileRows;                 // 8192
+constexpr size_t kCountersBytes = (size_t)kMaxTiles * sizeof(unsigned);
+constexpr size_t kHeaderBytes = kCountersBytes + 256;           // + error word, padded
+
 // Launch geometry of any4_linear for one shape on one device.
 struct LinearPlan {
-  int nt;               // n8 token tiles: 1 for M <= 8, 2 for M <= 16
-  int warps;            // warps that receive atoms (each gets >= 1)
-  int ctas;             // thread blocks
-  long long atoms;      // (N/16) * (K/64)
-  size_t counters_bytes;
+  long long units;      // tiles * chunks (one unit = 128 rows x 64 columns)
+  int ctas;             // persistent CTAs, one per SM at most
   size_t partials_bytes;
   size_t workspace_bytes;
-  size_t smem_bytes;    // dynamic shared memory per CTA
 };
-
-// The workspace starts with one arrival counter per possible 16-row tile, so
-// the counters of every shape live in the same zero-initialised header
-// whatever the shape of earlier calls; this bounds N at 16 * kMaxTiles rows.
-constexpr int kMaxTiles = 65536;
 
 LinearPlan plan_linear(int m, const Layout& L, int num_sms);
 

@@ -1,28 +1,38 @@
-// any4_linear: y = x . W_hat^T with W stored as any4 (per-row 16-entry bf16
-// table, 4-bit indices, per-group bf16 scale/offset).
+// any4_linear on B200 (sm_100a): y = x . W_hat^T with W stored as any4.
 //
-// Method: any4 explainer (10100.com, article 149119421) section 2 (per-row LUT,
-// index lookup at inference), section 2.1 (per-group alpha/beta), section 3
-// (table kept in registers, pre-arranged weights, batch 1-16 on tensor cores).
+// Method (any4 explainer, 10100.com article 149119421): every row of W has its
+// own table (LUT) of 16 bf16 values and every weight is a 4-bit index into it
+// (section 2); each contiguous group of G columns has a scale alpha and an
+// offset beta (section 2.1); w_hat = fma(alpha, LUT[idx], beta). tinygemm
+// (section 3) keeps the table next to the arithmetic and runs batch 1-16 on
+// the tensor cores; this kernel is a fresh design for Blackwell.
 //
-// Kernel structure (B200):
-//  * Work is the flat sequence of 512-byte atoms (16 rows x 64 columns) of the
-//    packed weight; atoms of consecutive tiles are contiguous, so a warp's share
-//    is one contiguous byte range that it streams with 128-bit loads, several
-//    atoms in flight.
-//  * Every warp gets an equal share (stream-K over atoms), so all SMs finish
-//    together whatever N and K are.
-//  * Decode: each lane keeps the low and high bytes of its two rows' tables in
-//    registers (16 registers) and looks up 4 indices at a time with byte
-//    permutes (2 lookups per byte plane + 1 select on index bit 3, then the
-//    bytes are interleaved into bf16 pairs). The group scale and offset are
-//    applied with one bf16x2 fma per pair, giving the operand of an m16n8k16
-//    bf16 tensor-core tile (weights as the 16-row side, tokens as the 8-wide
-//    side, fp32 accumulation).
-//  * A tile whose atoms are split between warps is finished by the last warp
-//    to arrive: each contributor stores its fp32 partial tile and bumps the
-//    tile's counter; the one that completes the count sums all partials in
-//    warp order (deterministic) and writes y. Nobody waits on anybody.
+// One persistent CTA per SM, 14 warps with fixed roles:
+//  * warps 0-7, two decoder warpgroups. Thread r of a warpgroup owns weight
+//    row r of the current 128-row tile, which is also Tensor Memory lane r.
+//    For every (tile, 64-column chunk) "unit" the warpgroup's threads read
+//    their row's 32 index bytes (one 512-byte coalesced load per warp and
+//    half), turn each byte -- the indices of two adjacent columns -- into a
+//    bf16 pair with ONE shared-memory load from a per-row pair table
+//    (256 entries: (LUT[lo nibble], LUT[hi nibble])), apply alpha/beta with
+//    one bf16x2 fma, and store the 64 weights of the row into a Tensor Memory
+//    operand buffer (tcgen05.st). The two warpgroups take alternate units.
+//  * warp 13 loads the matching 16 x 64 activation chunk with TMA (128-byte
+//    swizzle; rows past M are zero-filled by TMA).
+//  * warp 12 issues tcgen05.mma (M=128, N=16, K=16; A from Tensor Memory, B =
+//    activations from shared memory) accumulating fp32 in Tensor Memory.
+//  * warps 8-11 read the accumulator back at the end of each tile segment and
+//    write y (bf16) or, for a tile split between CTAs, an fp32 partial; the
+//    last CTA to finish a split tile sums the partials in CTA order (fixed,
+//    deterministic) and writes y. Nobody waits for another CTA.
+//  Stages hand over through mbarriers; every wait has a time limit after which
+//  the CTA records an error bit in the workspace, skips the remaining work and
+//  still releases its Tensor Memory.
+//
+// Work split: the units of all tiles form one sequence; CTA c gets an equal
+// contiguous share (stream-K), so every SM streams the same number of bytes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
 #include <atomic>
@@ -33,281 +43,535 @@ namespace any4 {
 
 namespace {
 
-constexpr int kWarpsPerCta = 8;
-constexpr int kCtasPerSm = 2;
-constexpr int kMinAtomsPerWarp = 4;
-constexpr int kPrefetch = 4;
-constexpr size_t kMaxSmemPerCta = 100 * 1024;   // keeps two CTAs per SM
+constexpr int kDecoderThreads = 256;       // warps 0-7
+constexpr int kEpilogueWarp0 = 8;          // warps 8-11
+constexpr int kMmaWarp = 12;
+constexpr int kThreads = 14 * 32;          // + warp 13: TMA
+constexpr int kAStages = 4;                // Tensor Memory operand buffers per warpgroup
+constexpr int kPrefetch = 4;               // units in flight per decoder thread (== kAStages)
+constexpr int kXStages = 8;                // activation chunks in shared memory
+constexpr int kTokens = 16;                // MMA N
+constexpr int kXStageBytes = kTokens * kChunkK * 2;   // 2048
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kDCol0 = 0;             // two 16-column fp32 accumulators
+constexpr uint32_t kACol0 = 32;            // 8 operand buffers of 32 columns
+constexpr uint32_t kACols = kChunkK / 2;
+constexpr uint32_t kTableAddr = 65536;     // shared-window address of the pair tables
+constexpr uint32_t kTableBlock = 65536;    // 256 entries x 64 rows x 4 bytes
+constexpr int kSmemBytes = 232448;         // 227 KB: the per-block maximum
+constexpr long long kWaitCycles = 4000000000ll;   // about 2 s, then give up
 
-struct LinearArgs {
-  const uint16_t* x;
+static_assert(kPrefetch == kAStages, "decoder ring slot doubles as operand slot");
+
+// tcgen05 instruction descriptor (kind::f16): D fp32, A and B bf16, both
+// K-major, N = 16, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            ((uint32_t)(kTokens >> 3) << 17) | ((uint32_t)(kTileRows >> 4) << 24);
+
+enum : unsigned {
+  kErrAEmpty = 1u, kErrAFull = 2u, kErrXEmpty = 4u, kErrXFull = 8u, kErrDEmpty = 16u,
+  kErrDFull = 32u, kErrSmem = 64u, kErrDrain = 128u
+};
+
+struct Params {
   const uint8_t* packed;
   uint16_t* y;
   float* partials;
   unsigned* counters;
-  Layout L;
-  int m;
-  int warps;
-  long long atoms;
+  unsigned* error;
+  int m, n, k, g;
+  int chunks, groups, gshift;
+  int ctas;
+  long long units;
+  size_t w_off, lut_off, ab_off;
 };
 
-// Warp that owns atom a under the split a_begin(w) = floor(w * A / W).
-__device__ __forceinline__ int warp_of_atom(long long a, long long A, int W) {
-  return (int)(((a + 1) * (long long)W - 1) / A);
+struct SmemCtl {
+  uint64_t a_full[2][kAStages];
+  uint64_t a_empty[2][kAStages];
+  uint64_t x_full[kXStages];
+  uint64_t x_empty[kXStages];
+  uint64_t d_full[2];
+  uint64_t d_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  unsigned ticket;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-// Decode one packed word (8 indices: 4 of row g in bits 0..15, 4 of row g+8 in
-// bits 16..31) into the four bf16x2 A-operand registers of the m16n8k16 tile.
-__device__ __forceinline__ void decode_word(uint32_t w, const uint32_t (&lo0)[4],
-                                            const uint32_t (&hi0)[4], const uint32_t (&lo1)[4],
-                                            const uint32_t (&hi1)[4], uint32_t (&a)[4]) {
-  const uint32_t w7 = w & 0x77777777u;                          // entry within a half table
-  const uint32_t sel = ((w >> 1) & 0x44444444u) | 0x32103210u;  // byte j of half (bit 3)
-  const uint32_t w7h = w7 >> 16, selh = sel >> 16;
-  {
-    const uint32_t pa = prmt(lo0[0], lo0[1], w7), pb = prmt(lo0[2], lo0[3], w7);
-    const uint32_t qa = prmt(hi0[0], hi0[1], w7), qb = prmt(hi0[2], hi0[3], w7);
-    const uint32_t lo = prmt(pa, pb, sel), hi = prmt(qa, qb, sel);
-    a[0] = prmt(lo, hi, 0x5140u);   // columns 2t, 2t+1
-    a[2] = prmt(lo, hi, 0x7362u);   // columns 2t+8, 2t+9
-  }
-  {
-    const uint32_t pa = prmt(lo1[0], lo1[1], w7h), pb = prmt(lo1[2], lo1[3], w7h);
-    const uint32_t qa = prmt(hi1[0], hi1[1], w7h), qb = prmt(hi1[2], hi1[3], w7h);
-    const uint32_t lo = prmt(pa, pb, selh), hi = prmt(qa, qb, selh);
-    a[1] = prmt(lo, hi, 0x5140u);
-    a[3] = prmt(lo, hi, 0x7362u);
-  }
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-template <int NT>
-__device__ __forceinline__ void store_tile(const LinearArgs& p, int tile, int lane,
-                                           const float (&acc)[NT][4]) {
-  const int g = lane >> 2, t = lane & 3;
-  const int n0 = tile * kTileRows + g;
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = 8 * j + 2 * t + (i & 1);
-      const int n = n0 + 8 * (i >> 1);
-      if (m < p.m) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(acc[j][i]);
-        p.y[(size_t)m * p.L.n + n] = *reinterpret_cast<const uint16_t*>(&h);
-      }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_st_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+      "%29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_x16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of one 16-token x 16-column activation slice:
+// K-major, 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t x_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Bounded wait on an mbarrier phase. Gives up (returns false) when the CTA is
+// already aborting, or after kWaitCycles, in which case it starts the abort.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         unsigned* err, unsigned code) {
+  if (*abort_flag) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      atomicOr(err, code);
+      return false;
     }
   }
 }
 
-// End of a warp's run over tile `tile` covering atoms [sb, se). Rarely taken
-// (at most once per tile a warp touches), so it is kept out of line to leave
-// the registers of the streaming loop alone.
-template <int NT>
-__device__ __noinline__ void finish_segment(const LinearArgs& p, int wid, int lane, int tile,
-                                               long long sb, long long se, long long a_begin,
-                                               const float (&acc)[NT][4]) {
-  const int KA = p.L.katoms;
-  const long long t0 = (long long)tile * KA, t1 = t0 + KA;
-  if (sb == t0 && se == t1) {          // the whole tile: no one else contributes
-    store_tile<NT>(p, tile, lane, acc);
+// CTA that owns unit u under the split U0(c) = floor(c * U / C).
+__device__ __forceinline__ int cta_of_unit(long long u, long long units, int ctas) {
+  return (int)(((u + 1) * (long long)ctas - 1) / units);
+}
+
+// ----------------------------------------------------------- pair tables
+
+// Build this warpgroup's half (entries 128*wg .. 128*wg+127) of the pair table
+// of row r: entry e = (LUT[e & 15], LUT[e >> 4]) as a bf16 pair, so the index
+// byte of two adjacent columns looks up both weights at once. `lut` holds the
+// row's 16 bf16 values as 8 pairs. Framed by decoder barriers so no thread
+// still reads the previous table and none reads this one half-built.
+__device__ __noinline__ void build_table(uint32_t row_base, const uint32_t* lut, int wg) {
+  named_bar_sync(1, kDecoderThreads);
+  uint32_t lo[8], hi[4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) lo[i] = lut[i];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) hi[h] = wg ? lo[4 + h] : lo[h];
+  const uint32_t addr0 = row_base + (uint32_t)wg * 128u * 256u;
+#pragma unroll
+  for (int i = 0; i < 128; ++i) {
+    const int lo_idx = i & 15, hi_idx = i >> 4;     // high nibble = 8 * wg + hi_idx
+    const uint32_t sel = ((lo_idx & 1) ? 0x32u : 0x10u) | (((hi_idx & 1) ? 0x76u : 0x54u) << 8);
+    sts32(addr0 + (uint32_t)i * 256u, prmt(lo[lo_idx >> 1], hi[hi_idx >> 1], sel));
+  }
+  named_bar_sync(1, kDecoderThreads);
+}
+
+__device__ __forceinline__ void load_lut(const Params& p, int tile, int r, uint32_t (&lut)[8]) {
+  const uint4* src = reinterpret_cast<const uint4*>(p.packed + p.lut_off +
+                                                    ((size_t)tile * kTileRows + r) * 32);
+  const uint4 a = ld_nc_v4(src), b = ld_nc_v4(src + 1);
+  lut[0] = a.x; lut[1] = a.y; lut[2] = a.z; lut[3] = a.w;
+  lut[4] = b.x; lut[5] = b.y; lut[6] = b.z; lut[7] = b.w;
+}
+
+// ------------------------------------------------------------------ kernel
+
+__global__ void __launch_bounds__(kThreads, 1)
+    linear_tc_kernel(const __grid_constant__ CUtensorMap tmap, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(base + kXStages * kXStageBytes);
+  const uint32_t x_addr0 = base_addr;
+
+  // The pair tables sit at a fixed shared address so one byte permute forms a
+  // lookup address; the ring and control block must fit below it.
+  if (smem_u32(ctl + 1) > kTableAddr || kTableAddr + 2 * kTableBlock > raw_addr + kSmemBytes) {
+    if (threadIdx.x == 0) atomicOr(p.error, kErrSmem);
     return;
   }
-  constexpr int kSlot = 32 * 4 * NT;   // floats per partial tile
-  const int slot = 2 * wid + ((long long)tile == a_begin / KA ? 0 : 1);
-  float* dst = p.partials + (size_t)slot * kSlot + lane * 4 * NT;
+
+  const long long U = p.units;
+  const long long U0 = (long long)blockIdx.x * U / p.ctas;
+  const long long U1 = (long long)(blockIdx.x + 1) * U / p.ctas;
+  const long long nunits = U1 - U0;
+  const int C = p.chunks;
+  const int t_first = (int)(U0 / C);
+  const int t_last = (int)((U1 - 1) / C);
+
+  volatile int* abort_flag = &ctl->abort_flag;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < 2; ++w)
+      for (int s = 0; s < kAStages; ++s) {
+        mbar_init(smem_u32(&ctl->a_full[w][s]), 4);    // one arrival per decoder warp
+        mbar_init(smem_u32(&ctl->a_empty[w][s]), 1);   // tcgen05.commit
+      }
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(smem_u32(&ctl->x_full[s]), 1);         // expect_tx arrival + bytes
+      mbar_init(smem_u32(&ctl->x_empty[s]), 1);        // tcgen05.commit
+    }
+    for (int d = 0; d < 2; ++d) {
+      mbar_init(smem_u32(&ctl->d_full[d]), 1);         // tcgen05.commit
+      mbar_init(smem_u32(&ctl->d_empty[d]), 4);        // one arrival per epilogue warp
+    }
+    mbar_init(smem_u32(&ctl->mma_done), 1);
+    ctl->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&ctl->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------ decoders
+    const int wg = warp >> 2, q = warp & 3, r = q * 32 + lane;
+    const uint32_t row_base = kTableAddr + (uint32_t)(r >> 6) * kTableBlock + 4u * (r & 63);
+    const uint32_t addr_bytes = (4u * (r & 63)) | ((1u + (uint32_t)(r >> 6)) << 16);
+    const uint32_t lane_tmem = tmem + ((uint32_t)(q * 32) << 16);
+    const uint8_t* wsrc = p.packed + p.w_off + (size_t)q * 1024 + (size_t)lane * 16;
+    const uint32_t* absrc = reinterpret_cast<const uint32_t*>(p.packed + p.ab_off) + r;
+
+    // the prefetch head walks this warpgroup's units (every second one)
+    long long up = U0 + wg;
+    int tile_p = (int)(up / C), chunk_p = (int)(up - (long long)tile_p * C);
+    uint4 v0[kPrefetch], v1[kPrefetch];
+    uint32_t ab[kPrefetch];
+    auto issue = [&](int s) {
+      const uint8_t* src = wsrc + (size_t)up * kUnitBytes;
+      v0[s] = ld_stream_v4(src);
+      v1[s] = ld_stream_v4(src + 512);
+      ab[s] = ld_nc_u32(absrc + ((size_t)tile_p * p.groups + (chunk_p >> p.gshift)) * kTileRows);
+      up += 2;
+      chunk_p += 2;
+      while (chunk_p >= C) { chunk_p -= C; ++tile_p; }
+    };
 #pragma unroll
-  for (int j = 0; j < NT; ++j)
-    __stcg(reinterpret_cast<float4*>(dst) + j, make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]));
-  __threadfence();
-  __syncwarp();
-  const int w_first = warp_of_atom(t0, p.atoms, p.warps);
-  const int w_last = warp_of_atom(t1 - 1, p.atoms, p.warps);
-  unsigned prev = 0;
-  if (lane == 0) prev = atomicAdd(p.counters + tile, 1u);
-  prev = __shfl_sync(0xffffffffu, prev, 0);
-  if (prev != (unsigned)(w_last - w_first)) return;   // not the last contributor
-  __threadfence();
-  float sum[NT][4];
+    for (int s = 0; s < kPrefetch; ++s)
+      if (up < U1) issue(s);
+
+    long long uc = U0 + wg;                        // unit being decoded
+    int tile_c = (int)(uc / C), chunk_c = (int)(uc - (long long)tile_c * C);
+    int built = t_first - 1;                       // last tile whose table is built
+    uint32_t lut_next[8];
+    load_lut(p, t_first, r, lut_next);
+
+    for (int n0 = 0;; n0 += kPrefetch) {
+      bool done = false;
 #pragma unroll
-  for (int j = 0; j < NT; ++j)
+      for (int s = 0; s < kPrefetch; ++s) {
+        if (uc >= U1) { done = true; break; }
+        while (built < tile_c) {
+          build_table(row_base, lut_next, wg);
+          ++built;
+          if (built < t_last) load_lut(p, built + 1, r, lut_next);
+        }
+        const uint4 a = v0[s], b = v1[s];
+        const uint32_t sab = ab[s];
+        if (up < U1) issue(s);
+        const uint32_t use = (uint32_t)(n0 / kPrefetch);
+        if (wait_bar(smem_u32(&ctl->a_empty[wg][s]), (use & 1u) ^ 1u, abort_flag, p.error,
+                     kErrAEmpty)) {
+          const uint32_t al = prmt(sab, sab, 0x1010u), be = prmt(sab, sab, 0x3232u);
+          const uint32_t words[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          uint32_t out[32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sum[j][i] = 0.0f;
-  // contributors in warp order, loads of a batch issued before they are summed
-  constexpr int kBatch = 4;
-  for (int w0 = w_first; w0 <= w_last; w0 += kBatch) {
-    float part[kBatch][NT][4];
+          for (int wi = 0; wi < 8; ++wi)
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      const int w = w0 + b;
-      if (w <= w_last) {
-        const long long wb = (long long)w * p.atoms / p.warps;
-        const int s = 2 * w + ((long long)tile == wb / KA ? 0 : 1);
-        const float4* src = reinterpret_cast<const float4*>(p.partials + (size_t)s * kSlot + lane * 4 * NT);
+            for (int bi = 0; bi < 4; ++bi) {
+              const uint32_t addr = prmt(words[wi], addr_bytes, 0x7604u | ((uint32_t)bi << 4));
+              out[wi * 4 + bi] = fma_bf16x2(lds32(addr), al, be);
+            }
+          tc_st_x32(lane_tmem + kACol0 + (uint32_t)(wg * kAStages + s) * kACols, out);
+          tc_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&ctl->a_full[wg][s]));
+        uc += 2;
+        chunk_c += 2;
+        while (chunk_c >= C) { chunk_c -= C; ++tile_c; }
+      }
+      if (done) break;
+    }
+    // both warpgroups build every tile's table, so their barriers pair up
+    while (built < t_last) {
+      build_table(row_base, lut_next, wg);
+      ++built;
+      if (built < t_last) load_lut(p, built + 1, r, lut_next);
+    }
+  } else if (warp < 12) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t lane_tmem = tmem + ((uint32_t)(q * 32) << 16);
+    for (int t = t_first; t <= t_last; ++t) {
+      const int s = t - t_first, d = s & 1;
+      const long long sb = max(U0, (long long)t * C), se = min(U1, (long long)(t + 1) * C);
+      uint32_t raw[16];
+      const bool ok = wait_bar(smem_u32(&ctl->d_full[d]), (uint32_t)(s >> 1) & 1u, abort_flag,
+                               p.error, kErrDFull);
+      if (ok) {
+        tc_fence_after();
+        tc_ld_x16(lane_tmem + kDCol0 + 16u * d, raw);
+        tc_wait_ld();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ctl->d_empty[d]));
+      float v[16];
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          const float4 v = __ldcg(src + j);
-          part[b][j][0] = v.x; part[b][j][1] = v.y; part[b][j][2] = v.z; part[b][j][3] = v.w;
+      for (int i = 0; i < 16; ++i) v[i] = ok ? __uint_as_float(raw[i]) : 0.0f;
+      const int n_row = t * kTileRows + r;
+      const bool full = sb == (long long)t * C && se == (long long)(t + 1) * C;
+      if (full) {
+        if (ok && n_row < p.n)
+          for (int m = 0; m < p.m; ++m) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(v[m]);
+            p.y[(size_t)m * p.n + n_row] = *reinterpret_cast<const uint16_t*>(&h);
+          }
+        continue;
+      }
+      // split tile: publish this CTA's fp32 partial (the token columns that
+      // exist); the last CTA to arrive sums them
+      const int nq = (p.m + 3) >> 2;
+      const int my_slot = 2 * blockIdx.x + (t == t_first ? 0 : 1);
+      float4* dst = reinterpret_cast<float4*>(p.partials + ((size_t)my_slot * kTileRows + r) * 16);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (i < nq) __stcg(dst + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+      __threadfence();
+      named_bar_sync(2, 128);
+      if (warp == kEpilogueWarp0 && lane == 0) ctl->ticket = atomicAdd(p.counters + t, 1u);
+      named_bar_sync(2, 128);
+      const int c_first = cta_of_unit((long long)t * C, U, p.ctas);
+      const int c_last = cta_of_unit((long long)(t + 1) * C - 1, U, p.ctas);
+      if (ctl->ticket != (unsigned)(c_last - c_first)) continue;
+      __threadfence();
+      float acc[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = 0.0f;
+      // contributors in CTA order; a batch's loads are all issued before it is summed
+      constexpr int kBatch = 8;
+      for (int i = 0; i < nq; ++i)
+        for (int c0 = c_first; c0 <= c_last; c0 += kBatch) {
+          float4 f[kBatch];
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            const int c = c0 + b;
+            f[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c <= c_last) {
+              const long long cu0 = (long long)c * U / p.ctas;
+              const int slot = 2 * c + ((long long)t == cu0 / C ? 0 : 1);
+              f[b] = __ldcg(reinterpret_cast<const float4*>(
+                                p.partials + ((size_t)slot * kTileRows + r) * 16) + i);
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < kBatch; ++b) {
+            acc[4 * i] += f[b].x; acc[4 * i + 1] += f[b].y;
+            acc[4 * i + 2] += f[b].z; acc[4 * i + 3] += f[b].w;
+          }
+        }
+      if (n_row < p.n && !*abort_flag)
+        for (int m = 0; m < p.m; ++m) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(acc[m]);
+          p.y[(size_t)m * p.n + n_row] = *reinterpret_cast<const uint16_t*>(&h);
+        }
+      if (warp == kEpilogueWarp0 && lane == 0) p.counters[t] = 0u;   // ready for the next call
+    }
+  } else if (warp == kMmaWarp) {
+    // ----------------------------------------------------------------- MMA
+    if (lane == 0) {
+      long long j = 0;
+      for (int t = t_first; t <= t_last; ++t) {
+        const int s = t - t_first, d = s & 1;
+        const long long se = min(U1, (long long)(t + 1) * C);
+        wait_bar(smem_u32(&ctl->d_empty[d]), ((uint32_t)(s >> 1) & 1u) ^ 1u, abort_flag, p.error,
+                 kErrDEmpty);
+        tc_fence_after();
+        bool first = true;
+        for (; U0 + j < se; ++j) {
+          const int wg = (int)(j & 1), slot = (int)((j >> 1) & (kAStages - 1));
+          const uint32_t use = (uint32_t)(j >> 3);
+          const int xs = (int)(j & (kXStages - 1));
+          const bool ok =
+              wait_bar(smem_u32(&ctl->a_full[wg][slot]), use & 1u, abort_flag, p.error, kErrAFull) &&
+              wait_bar(smem_u32(&ctl->x_full[xs]), (uint32_t)(j >> 3) & 1u, abort_flag, p.error,
+                       kErrXFull);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t a_col = tmem + kACol0 + (uint32_t)(wg * kAStages + slot) * kACols;
+            const uint64_t desc = x_desc(x_addr0 + (uint32_t)xs * kXStageBytes);
+#pragma unroll
+            for (int i = 0; i < kChunkK / 16; ++i)
+              tc_mma(tmem + kDCol0 + 16u * d, a_col + 8u * i, desc + 2u * i,
+                     (first && i == 0) ? 0u : 1u);
+            first = false;
+          }
+          tc_commit(smem_u32(&ctl->a_empty[wg][slot]));
+          tc_commit(smem_u32(&ctl->x_empty[xs]));
+        }
+        tc_commit(smem_u32(&ctl->d_full[d]));
+      }
+      // every MMA has completed before Tensor Memory is released
+      tc_commit(smem_u32(&ctl->mma_done));
+      const long long t0 = clock64();
+      while (!mbar_try_wait(smem_u32(&ctl->mma_done), 0)) {
+        if (clock64() - t0 > kWaitCycles) { atomicOr(p.error, kErrDrain); break; }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int chunk = (int)(U0 - (long long)t_first * C);
+      int last_use[kXStages];
+#pragma unroll
+      for (int s = 0; s < kXStages; ++s) last_use[s] = -1;
+      for (long long j = 0; j < nunits; ++j) {
+        const int xs = (int)(j & (kXStages - 1));
+        const uint32_t use = (uint32_t)(j >> 3);
+        if (wait_bar(smem_u32(&ctl->x_empty[xs]), (use & 1u) ^ 1u, abort_flag, p.error, kErrXEmpty)) {
+          mbar_arrive_expect_tx(smem_u32(&ctl->x_full[xs]), kXStageBytes);
+          tma_load_2d(x_addr0 + (uint32_t)xs * kXStageBytes, &tmap, chunk * kChunkK, 0,
+                      smem_u32(&ctl->x_full[xs]));
+          last_use[xs] = (int)use;
+        }
+        if (++chunk == C) chunk = 0;
+      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (int s = 0; s < kXStages; ++s) {
+        if (last_use[s] < 0) continue;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(smem_u32(&ctl->x_full[s]), (uint32_t)last_use[s] & 1u)) {
+          if (clock64() - t0 > kWaitCycles) { atomicOr(p.error, kErrDrain); break; }
         }
       }
     }
-#pragma unroll
-    for (int b = 0; b < kBatch; ++b)
-      if (w0 + b <= w_last)
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) sum[j][i] += part[b][j][i];
   }
-  store_tile<NT>(p, tile, lane, sum);
-  if (lane == 0) p.counters[tile] = 0u;   // ready for the next call
-}
 
-template <int NT>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) linear_kernel(const LinearArgs p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int lane = threadIdx.x & 31;
-  const int wid = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
-  const long long A = p.atoms;
-  const int KA = p.L.katoms, K = p.L.k, G = p.L.g, NG = p.L.groups;
-  const int atoms_per_group = G / kAtomK;
-
-  // ---- this CTA's atom range, and the tables / scales it covers
-  const int w_lo = blockIdx.x * kWarpsPerCta;
-  const int w_hi = min(w_lo + kWarpsPerCta, p.warps) - 1;
-  const long long cta_a0 = (long long)w_lo * A / p.warps;
-  const long long cta_a1 = (long long)(w_hi + 1) * A / p.warps;
-  const int t_lo = (int)(cta_a0 / KA);
-  const int t_hi = (int)((cta_a1 - 1) / KA);
-  const long long rec_lo = (long long)t_lo * NG + (int)(cta_a0 - (long long)t_lo * KA) / atoms_per_group;
-  const long long rec_hi = (long long)t_hi * NG + (int)(cta_a1 - 1 - (long long)t_hi * KA) / atoms_per_group;
-  const int lut_bytes = (t_hi - t_lo + 1) * kTileRows * 32;
-  uint8_t* s_lut = smem;
-  uint32_t* s_ab = reinterpret_cast<uint32_t*>(smem + lut_bytes);
-
-  const bool active = wid < p.warps;
-  const long long a_begin = active ? (long long)wid * A / p.warps : 0;
-  const long long a_end = active ? (long long)(wid + 1) * A / p.warps : 0;
-  const uint8_t* wsec = p.packed + p.L.w_off + (size_t)lane * 16;
-
-  // weights first: the first atoms are in flight while the tables are staged
-  uint4 buf[kPrefetch];
-#pragma unroll
-  for (int j = 0; j < kPrefetch; ++j)
-    if (a_begin + j < a_end) buf[j] = ld_stream_v4(wsec + (size_t)(a_begin + j) * kAtomBytes);
-
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(p.packed + p.L.lut_off + (size_t)t_lo * kTileRows * 32);
-    uint4* dst = reinterpret_cast<uint4*>(s_lut);
-    for (int i = threadIdx.x; i < lut_bytes / 16; i += blockDim.x) dst[i] = __ldg(src + i);
-    const uint4* asrc = reinterpret_cast<const uint4*>(p.packed + p.L.ab_off) + rec_lo * 4;
-    uint4* adst = reinterpret_cast<uint4*>(s_ab);
-    const int nrec4 = (int)(rec_hi - rec_lo + 1) * 4;   // 16 rows x u32 = 4 x uint4 per record
-    for (int i = threadIdx.x; i < nrec4; i += blockDim.x) adst[i] = __ldg(asrc + i);
-  }
+  tc_fence_before();
   __syncthreads();
-  if (!active) return;
-
-  const int g = lane >> 2, t = lane & 3;
-  // x rows feeding this lane's B fragments (token 8j+g). Columns of tokens
-  // >= M repeat token M-1; their outputs are never stored.
-  const uint32_t* xrow[NT];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int m = min(8 * j + g, p.m - 1);
-    xrow[j] = reinterpret_cast<const uint32_t*>(p.x + (size_t)m * K) + t;
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
   }
-  // B fragments of one atom: [j][step][b0, b1]; c = first column / 2 of the atom
-  uint32_t xf[2][NT][4][2];
-  auto load_x = [&](int c, uint32_t (&dst)[NT][4][2]) {
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        dst[j][s][0] = __ldg(xrow[j] + c + 8 * s);
-        dst[j][s][1] = __ldg(xrow[j] + c + 8 * s + 4);
-      }
-  };
-
-  // Position of the current atom, advanced incrementally (no divisions in the loop).
-  int tile = (int)(a_begin / KA);
-  int ka = (int)(a_begin - (long long)tile * KA);   // atom within the tile
-  int grp = ka / atoms_per_group;
-  int kg = ka - grp * atoms_per_group;               // atom within the group
-  load_x(ka * (kAtomK / 2), xf[0]);
-
-  float acc[NT][4];
-  uint32_t lo0[4], hi0[4], lo1[4], hi1[4];
-  uint32_t al0 = 0, be0 = 0, al1 = 0, be1 = 0;
-  int cur_tile = -1;
-  long long seg_begin = a_begin;
-
-  for (long long a0 = a_begin; a0 < a_end; a0 += kPrefetch) {
-#pragma unroll
-    for (int jj = 0; jj < kPrefetch; ++jj) {
-      const long long a = a0 + jj;
-      if (a >= a_end) break;
-      const uint4 wv = buf[jj];
-      if (a + kPrefetch < a_end) buf[jj] = ld_stream_v4(wsec + (size_t)(a + kPrefetch) * kAtomBytes);
-      // kPrefetch is even, so jj's parity is the atom's parity within the run
-      uint32_t (&xc)[NT][4][2] = xf[jj & 1];
-      const int ka_next = ka + 1 == KA ? 0 : ka + 1;
-      if (a + 1 < a_end) load_x(ka_next * (kAtomK / 2), xf[(jj + 1) & 1]);
-
-      if (tile != cur_tile) {
-        if (cur_tile >= 0) finish_segment<NT>(p, wid, lane, cur_tile, seg_begin, a, a_begin, acc);
-        const uint4* r0 = reinterpret_cast<const uint4*>(s_lut + ((tile - t_lo) * kTileRows + g) * 32);
-        const uint4* r1 = r0 + 16;   // row g+8 is 8 rows * 32 bytes further
-        const uint4 l0 = r0[0], h0 = r0[1], l1 = r1[0], h1 = r1[1];
-        lo0[0] = l0.x; lo0[1] = l0.y; lo0[2] = l0.z; lo0[3] = l0.w;
-        hi0[0] = h0.x; hi0[1] = h0.y; hi0[2] = h0.z; hi0[3] = h0.w;
-        lo1[0] = l1.x; lo1[1] = l1.y; lo1[2] = l1.z; lo1[3] = l1.w;
-        hi1[0] = h1.x; hi1[1] = h1.y; hi1[2] = h1.z; hi1[3] = h1.w;
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) acc[j][i] = 0.0f;
-        cur_tile = tile;
-        seg_begin = a;
-      }
-      if (kg == 0 || a == a_begin) {
-        const uint32_t* sr = s_ab + ((long long)tile * NG + grp - rec_lo) * kTileRows + g;
-        const uint32_t s0 = sr[0], s1 = sr[8];
-        al0 = prmt(s0, s0, 0x1010u); be0 = prmt(s0, s0, 0x3232u);   // (alpha, alpha), (beta, beta)
-        al1 = prmt(s1, s1, 0x1010u); be1 = prmt(s1, s1, 0x3232u);
-      }
-      const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        uint32_t af[4];
-        decode_word(words[s], lo0, hi0, lo1, hi1, af);
-        af[0] = fma_bf16x2(af[0], al0, be0);
-        af[2] = fma_bf16x2(af[2], al0, be0);
-        af[1] = fma_bf16x2(af[1], al1, be1);
-        af[3] = fma_bf16x2(af[3], al1, be1);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) mma_m16n8k16(acc[j], af, xc[j][s][0], xc[j][s][1]);
-      }
-      // advance to the next atom
-      if (++kg == atoms_per_group) { kg = 0; ++grp; }
-      ka = ka_next;
-      if (ka == 0) { ++tile; grp = 0; kg = 0; }
-    }
-  }
-  if (cur_tile >= 0) finish_segment<NT>(p, wid, lane, cur_tile, seg_begin, a_end, a_begin, acc);
 }
 
-// Dynamic shared memory of one CTA: the LUTs of the tiles and the scale
-// records of the groups its atom range touches (bounded by the widest CTA).
-size_t linear_smem_bytes(const Layout& L, long long atoms, int warps) {
-  const long long per_warp = (atoms + warps - 1) / warps;
-  const long long per_cta = per_warp * kWarpsPerCta + 1;
-  const long long tiles = per_cta / L.katoms + 2;
-  const long long recs = per_cta * kAtomK / L.g + 2;
-  return (size_t)(tiles * kTileRows * 32 + recs * kTileRows * 4);
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> fn{nullptr};
+  void* f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn.store(f, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
 }
 
-// Opt the kernels in to more than 48 KB of dynamic shared memory (once per
-// device; the attribute is per function and device).
 cudaError_t allow_large_smem() {
   static std::atomic<unsigned long long> done_mask{0};
   int dev = 0;
@@ -315,11 +579,7 @@ cudaError_t allow_large_smem() {
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (done_mask.load(std::memory_order_relaxed) & bit) return cudaSuccess;
-  e = cudaFuncSetAttribute(linear_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kMaxSmemPerCta);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(linear_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kMaxSmemPerCta);
+  e = cudaFuncSetAttribute(linear_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_relaxed);
   return e;
 }
@@ -327,44 +587,53 @@ cudaError_t allow_large_smem() {
 }  // namespace
 
 LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
+  (void)m;
   LinearPlan pl{};
-  pl.nt = m > 8 ? 2 : 1;
-  pl.atoms = (long long)L.tiles * L.katoms;
-  long long w = pl.atoms / kMinAtomsPerWarp;
-  const long long cap = (long long)num_sms * kCtasPerSm * kWarpsPerCta;
-  if (w > cap) w = cap;
-  if (w < 1) w = 1;
-  pl.warps = (int)w;
-  pl.ctas = (pl.warps + kWarpsPerCta - 1) / kWarpsPerCta;
-  pl.counters_bytes = (size_t)kMaxTiles * sizeof(unsigned);   // same for every shape
-  pl.partials_bytes = align_up((size_t)2 * pl.warps * 32 * 4 * pl.nt * sizeof(float), kAlign);
-  pl.workspace_bytes = pl.counters_bytes + pl.partials_bytes;
-  pl.smem_bytes = linear_smem_bytes(L, pl.atoms, pl.warps);
+  pl.units = (long long)L.tiles * L.chunks;
+  long long c = pl.units / 2;                  // at least two units per CTA
+  if (c > num_sms) c = num_sms;
+  if (c < 1) c = 1;
+  pl.ctas = (int)c;
+  pl.partials_bytes = (size_t)2 * pl.ctas * kTileRows * 16 * sizeof(float);
+  pl.workspace_bytes = kHeaderBytes + pl.partials_bytes;
   return pl;
 }
 
 cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout& L, int m,
                           uint16_t* y, void* workspace, const LinearPlan& plan,
                           cudaStream_t stream) {
-  LinearArgs p{};
-  p.x = x;
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return cudaErrorNotSupported;
+  cudaError_t e = allow_large_smem();
+  if (e != cudaSuccess) return e;
+
+  // activations: K x M bf16 (inner dimension first), 64 x 16 boxes, 128-byte
+  // swizzle; rows past M read as zero.
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)L.k, (cuuint64_t)m};
+  const cuuint64_t strides[1] = {(cuuint64_t)L.k * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kChunkK, (cuuint32_t)kTokens};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  Params p{};
   p.packed = packed;
   p.y = y;
-  p.counters = reinterpret_cast<unsigned*>(workspace);
-  p.partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + plan.counters_bytes);
-  p.L = L;
-  p.m = m;
-  p.warps = plan.warps;
-  p.atoms = plan.atoms;
-  const dim3 block(kWarpsPerCta * 32);
-  const size_t smem = linear_smem_bytes(L, plan.atoms, plan.warps);
-  if (smem > kMaxSmemPerCta) return cudaErrorInvalidValue;
-  cudaError_t e = smem > 48 * 1024 ? allow_large_smem() : cudaSuccess;
-  if (e != cudaSuccess) return e;
-  if (plan.nt == 1)
-    linear_kernel<1><<<plan.ctas, block, smem, stream>>>(p);
-  else
-    linear_kernel<2><<<plan.ctas, block, smem, stream>>>(p);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  p.counters = reinterpret_cast<unsigned*>(ws);
+  p.error = reinterpret_cast<unsigned*>(ws + kCountersBytes);
+  p.partials = reinterpret_cast<float*>(ws + kHeaderBytes);
+  p.m = m; p.n = L.n; p.k = L.k; p.g = L.g;
+  p.chunks = L.chunks; p.groups = L.groups;
+  p.gshift = 0;
+  while ((kChunkK << p.gshift) < L.g) ++p.gshift;
+  p.ctas = plan.ctas;
+  p.units = plan.units;
+  p.w_off = L.w_off; p.lut_off = L.lut_off; p.ab_off = L.ab_off;
+  linear_tc_kernel<<<plan.ctas, kThreads, kSmemBytes, stream>>>(tmap, p);
   return cudaGetLastError();
 }
 

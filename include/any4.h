@@ -62,7 +62,7 @@ typedef enum {
 /*
  * Size in bytes of the device-layout buffer any4_pack writes for an N x K
  * weight with group size G; 0 if the shape is not accepted. With Np = N
- * rounded up to a multiple of 128 (the padding rows are zeros), the size is
+ * rounded up to a multiple of 32 (the padding rows are zeros), the size is
  * Np*K/2 (indices) + 32*Np (LUT) + 4*Np*(K/G) (alpha and beta), each section
  * padded to 256 bytes. At K = 4096 the LUT adds 16*16/4096 = 0.0625 bit per
  * weight (explainer section 2.3).
@@ -100,9 +100,9 @@ ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t*
 /*
  * Bytes of workspace any4_linear needs for this shape on the CURRENT device
  * (the launch is sized by the device's SM count); 0 if the shape is not
- * accepted. The workspace holds a fixed header of 8192 arrival counters (one
- * per possible 128-row tile) and one error word, then the fp32 partial sums
- * of output tiles split along K between thread blocks.
+ * accepted. The workspace holds a fixed header of 65536 arrival counters (one
+ * per possible 16-row tile) and a reserved 256-byte area, then the fp32
+ * partial sums of output blocks split along K between thread blocks.
  */
 ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 
@@ -122,11 +122,10 @@ ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
  *
  * Each weight is dequantized as w_hat = fma(alpha, LUT[idx], beta) in bf16
  * (fma.rn.bf16x2: the exact value rounded once to bf16) and contracted on the
- * tensor cores (tcgen05) with fp32 accumulation; the fp32 result is rounded
- * to bf16 nearest-even. Tiles split along K are reduced in a fixed order, so
- * the result is deterministic. If an internal pipeline wait ever times out
- * (about 2 s) the kernel stops, leaves y incomplete and sets a nonzero error
- * word in the workspace header (byte offset 32768).
+ * tensor cores (mma.sync m16n8k16) with fp32 accumulation; the fp32 result
+ * is rounded to bf16 nearest-even. Blocks split along K are reduced in a
+ * fixed order, so the result is deterministic. No thread block ever waits on
+ * another one.
  */
 ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);

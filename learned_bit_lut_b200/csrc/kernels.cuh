@@ -17,18 +17,19 @@ cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint1
 cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream);
 
-// The workspace of any4_linear starts with one arrival counter per possible
-// 128-row tile, so the counters of every shape live in the same zero-filled
-// header whatever the shape of earlier calls; then one error word; then the
-// fp32 partial tiles.
-constexpr int kMaxTiles = kMaxRows / kTileRows;                 // 8192
+// The workspace of any4_linear starts with a fixed header of arrival
+// counters (one per possible 16-row tile, so the counters of every shape live
+// in the same zero-filled header whatever the shape of earlier calls), then a
+// reserved 256-byte word area, then the fp32 partial tiles.
+constexpr int kMaxTiles = kMaxRows / kTileRows;                 // 65536
 constexpr size_t kCountersBytes = (size_t)kMaxTiles * sizeof(unsigned);
-constexpr size_t kHeaderBytes = kCountersBytes + 256;           // + error word, padded
+constexpr size_t kHeaderBytes = kCountersBytes + 256;
 
 // Launch geometry of any4_linear for one shape on one device.
 struct LinearPlan {
-  long long units;      // tiles * chunks (one unit = 128 rows x 64 columns)
-  int ctas;             // persistent CTAs, one per SM at most
+  int nt;               // 8-token MMA column tiles: 1 for M <= 8, 2 for M <= 16
+  long long atoms;      // 32-row blocks x K/64
+  int ctas;             // persistent thread blocks
   size_t partials_bytes;
   size_t workspace_bytes;
 };

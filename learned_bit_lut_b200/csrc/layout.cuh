@@ -1,25 +1,32 @@
 // Device layout of a packed any4 weight (written by any4_pack).
 //
 // The explainer's tinygemm notes (10100.com, article 149119421, section 3) keep
-// the table close to the arithmetic and pre-arrange the weights in the compute
-// format. This layout is built for the B200 linear kernel of this library, in
-// which each decoder thread owns one weight row (one Tensor Memory lane):
+// the table next to the arithmetic and pre-arrange the weights in the compute
+// format. This layout is built for the operand layout of the m16n8k16 bf16
+// tensor-core tile used by the linear kernel of this library:
 //
-//  * rows are grouped in tiles of 128 (N is padded up with zero rows);
-//  * K is cut into chunks of 64 columns; one (tile, chunk) "unit" is 4096
-//    contiguous bytes, and units are stored tile by tile, chunk by chunk, so
-//    any run of consecutive units is one contiguous byte range;
-//  * inside a unit, warp quarter q (rows 32q..32q+31) owns 1024 bytes: first
-//    the 16 bytes of columns 0..31 of each of its 32 rows, then the 16 bytes of
-//    columns 32..63. A row's 16 bytes are its canonical index bytes (byte j
-//    holds columns 2j and 2j+1, low nibble first), so a warp reads 512
-//    contiguous bytes per 128-bit load.
+//  * rows are grouped in 16-row tiles (N is padded with zero rows up to a
+//    multiple of 32, so tiles pair up into 32-row blocks);
+//  * K is cut into 64-column "atoms"; an atom of a tile is 512 contiguous
+//    bytes, 16 per lane of a warp, so a warp streams it with one 128-bit load
+//    per lane; atoms of a tile follow each other, then the next tile;
+//  * inside an atom, lane (g = lane/4, t = lane%4) owns, for each of the four
+//    tensor-core steps s, one 32-bit word (c = 64*atom + 16*t + 4*s):
+//        bits  0..7   idx[row g  ][c], idx[row g  ][c+1]      (low nibble = c)
+//        bits  8..15  idx[row g  ][c+2], idx[row g  ][c+3]
+//        bits 16..23  idx[row g+8][c], idx[row g+8][c+1]
+//        bits 24..31  idx[row g+8][c+2], idx[row g+8][c+3]
+//    Every byte is one (even, odd) column pair of the canonical nibble layout.
+//    The m16n8k16 tile's columns 2t, 2t+1 | 2t+8, 2t+9 of step s are mapped
+//    to weight columns c, c+1 | c+2, c+3: a permutation of K inside the atom,
+//    applied identically to the activations, chosen so that the 16
+//    activation columns a lane needs over the four steps, 64*atom+16*t ..
+//    +15, are contiguous (two 128-bit loads).
 //
-// Sections (each starts on a 256-byte boundary):
-//   weights  [tiles][chunks][4 quarters][2 halves][32 rows][16 B]   Np*K/2 bytes
-//   lut      [Np rows][16 x bf16]  (canonical order)               32*Np bytes
-//   scales   [tiles][K/G groups][128 rows] u32 = alpha | beta << 16 4*Np*K/G bytes
-// with Np = N rounded up to a multiple of 128.
+// Sections (each starts on a 256-byte boundary), Np = N rounded up to 32:
+//   weights  [Np/16 tiles][K/64 atoms][32 lanes][4 x u32]      Np*K/2 bytes
+//   lut      [Np rows][16 x bf16]  (canonical order)             32*Np bytes
+//   scales   [Np/16 tiles][K/G groups][16 rows] u32 = alpha | beta << 16
 #pragma once
 
 #include <cstddef>
@@ -27,17 +34,18 @@
 
 namespace any4 {
 
-constexpr int kTileRows = 128;
-constexpr int kChunkK = 64;
-constexpr int kUnitBytes = kTileRows * kChunkK / 2;   // 4096
+constexpr int kTileRows = 16;
+constexpr int kBlockRows = 32;     // two tiles share one activation fragment
+constexpr int kAtomK = 64;
+constexpr int kAtomBytes = 512;
 constexpr int kAlign = 256;
 constexpr int kMaxRows = 1 << 20;
 
 struct Layout {
   int n, k, g;
-  int n_pad;        // n rounded up to a multiple of 128
-  int tiles;        // n_pad / 128
-  int chunks;       // k / 64
+  int n_pad;        // n rounded up to a multiple of 32
+  int tiles;        // n_pad / 16
+  int katoms;       // k / 64
   int groups;       // k / g
   size_t w_off, lut_off, ab_off, total;
 };
@@ -46,7 +54,7 @@ __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a -
 
 inline bool shape_ok(int n, int k, int g) {
   if (n <= 0 || k <= 0 || n > kMaxRows) return false;
-  if (n % 16 || k % kChunkK) return false;
+  if (n % 16 || k % kAtomK) return false;
   if (!(g == 64 || g == 128 || g == 256 || g == 512 || g == 1024)) return false;
   return k % g == 0;
 }
@@ -54,9 +62,9 @@ inline bool shape_ok(int n, int k, int g) {
 inline Layout make_layout(int n, int k, int g) {
   Layout L{};
   L.n = n; L.k = k; L.g = g;
-  L.n_pad = (int)align_up((size_t)n, kTileRows);
+  L.n_pad = (int)align_up((size_t)n, kBlockRows);
   L.tiles = L.n_pad / kTileRows;
-  L.chunks = k / kChunkK;
+  L.katoms = k / kAtomK;
   L.groups = k / g;
   L.w_off = 0;
   L.lut_off = align_up((size_t)L.n_pad * k / 2, kAlign);

@@ -30,9 +30,9 @@ def test_packed_bytes_accounting():
     idx, lut, ab = n * k // 2, 32 * n, 4 * n * (k // g)
     assert total == idx + lut + ab            # all sections already 256-byte multiples here
     assert lut * 8 / (n * k) == 0.0625        # explainer section 2.3
-    # N is padded to 128 rows; each section is rounded up to 256 bytes
-    assert a4.any4_packed_bytes(16, 64, 64) == 128 * 32 + 128 * 32 + 128 * 4
-    assert a4.any4_packed_bytes(144, 128, 64) == 256 * 64 + 256 * 32 + 256 * 2 * 4
+    # N is padded to 32 rows; each section is rounded up to 256 bytes
+    assert a4.any4_packed_bytes(16, 64, 64) == 32 * 32 + 32 * 32 + 256
+    assert a4.any4_packed_bytes(144, 128, 64) == 160 * 64 + 160 * 32 + 160 * 2 * 4
 
 
 @pytest.mark.parametrize("n,k,g", [(0, 64, 64), (15, 64, 64), (16, 63, 64), (16, 64, 32),

@@ -316,6 +316,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         del g
 
 
+def run_one(n: int, k: int, m: int, g: int, calls: int = 8):
+    """A few any4_linear calls of one shape (4 weight copies in rotation), for
+    profiler captures of a single launch."""
+    import torch
+
+    import learned_bit_lut_b200 as a4
+    dev = torch.device("cuda:0")
+    idx, lut, al, be = synth.random_any4(n, k, g, 0, layer="one")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+    ws = [a4.any4_pack(t(idx), t(lut), t(al), t(be), g) for _ in range(4)]
+    s = synth.channel_scale(k, 0, layer="one")
+    x = torch.from_numpy(synth.activations_bf16(m, s, 0, layer="one").view(np.int16)).to(dev).view(torch.bfloat16)
+    for i in range(calls):
+        a4.any4_linear(x, ws[i % 4], n, k, g)
+    torch.cuda.synchronize()
+    print(f"ran {calls} calls of N={n} K={k} M={m} G={g}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -325,7 +343,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--one", type=int, nargs=4, metavar=("N", "K", "M", "G"),
+                    help="only run a few calls of one shape (profiler captures)")
     args = ap.parse_args()
+    if args.one:
+        run_one(*args.one)
+        return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))

@@ -18,18 +18,22 @@ cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream);
 
 // The workspace of any4_linear starts with a fixed header of arrival
-// counters (one per possible 16-row tile, so the counters of every shape live
-// in the same zero-filled header whatever the shape of earlier calls), then a
-// reserved 256-byte word area, then the fp32 partial tiles.
+// counters (one per possible 32-row panel, so the counters of every shape live
+// in the same zero-filled header whatever the shape of earlier calls; sized for
+// 16-row tiles, which leaves room), then a reserved 256-byte word area whose
+// first word is the device status (0, or kStatusWaitTimeout when a kernel gave
+// up waiting for one of its own copies), then the fp32 partial sums.
 constexpr int kMaxTiles = kMaxRows / kTileRows;                 // 65536
 constexpr size_t kCountersBytes = (size_t)kMaxTiles * sizeof(unsigned);
 constexpr size_t kHeaderBytes = kCountersBytes + 256;
+constexpr unsigned kStatusWaitTimeout = 1u;
 
 // Launch geometry of any4_linear for one shape on one device.
 struct LinearPlan {
-  int nt;               // 8-token MMA column tiles: 1 for M <= 8, 2 for M <= 16
-  long long atoms;      // 32-row blocks x K/64
-  int ctas;             // persistent thread blocks
+  int mode;             // 0: M <= 4, 1: M <= 8 (row-pair operands); 2: M <= 16 (row operands)
+  int nf;               // fp32 results per lane and panel
+  long long units;      // panels x K/64 chunks
+  int ctas;             // persistent thread blocks (one per SM at most)
   size_t partials_bytes;
   size_t workspace_bytes;
 };

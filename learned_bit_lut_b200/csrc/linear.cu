@@ -5,35 +5,39 @@
 // (section 2); each contiguous group of G columns has a scale alpha and an
 // offset beta (section 2.1); w_hat = fma(alpha, LUT[idx], beta). tinygemm
 // (section 3) keeps the table next to the arithmetic and runs batch 1-16 on
-// the tensor cores. This kernel is designed from B200 measurements:
+// the tensor cores. This kernel is built from B200 measurements:
 //
-//  * Contraction: mma.sync m16n8k16 (bf16 in, fp32 accumulate), weights as
-//    the 16-row operand, tokens as the 8-wide one (two of them for M > 8).
-//    For this skinny shape it consumes ~128 weights per clock per SM, where a
-//    tcgen05.mma of 128 x 16 x 16 costs ~198 cycles whatever N is (~10
-//    weights per clock per SM), so the narrow-N path is the faster one here.
-//  * Decode, split across two pipes. In the m16n8k16 operand a lane holds 4
-//    weights of row g and 4 of row g+8 of a 16-row tile:
-//      - row g: byte permutes from the row's table held in registers as a
-//        low-byte and a high-byte plane (two 8-entry halves per plane, one
-//        select on index bit 3, one interleave): integer pipe only;
-//      - row g+8: each index byte (two adjacent columns) picks a bf16 pair
-//        from a 256-entry pair table (LUT[lo nibble], LUT[hi nibble]) in
-//        shared memory with one load; the byte permute that forms the address
-//        is the only integer op. Four bank copies per row make every warp-wide
-//        lookup conflict free.
-//    alpha/beta are applied with one bf16x2 fma per pair (w_hat rounded once
-//    to bf16), then the tile goes to the tensor core.
-//  * A thread block works on 32-row blocks (two 16-row tiles, so every
-//    activation fragment serves two MMAs); its 8 warps split the block's K
-//    range and share the pair tables; the fp32 tiles are summed across warps
-//    in shared memory in a fixed order.
-//  * Stream-K: the (block, 64-column atom) sequence is cut into equal
-//    contiguous shares, one per thread block (two blocks per SM). A block
-//    split between thread blocks is finished by the last one to arrive: each
-//    publishes an fp32 partial and bumps the block's counter; the last sums
-//    all partials in thread-block order (deterministic) and writes y. Nothing
-//    waits on another thread block.
+//  * Contraction: mma.sync m16n8k16 (bf16 in, fp32 accumulate). For M <= 16
+//    it consumes up to ~128 weights per clock per SM, where one tcgen05.mma of
+//    128 x N x 16 costs ~198 cycles whatever N is (~10 weights per clock per
+//    SM at this N), so the narrow-N path is the faster one for decode.
+//  * Decode: a shared-memory load is the only per-lane gather on the SM. Each
+//    index byte of the layout (layout.cuh) holds the indices of rows r and
+//    r+16 at one column and selects one bf16 pair (LUT_r[lo], LUT_r+16[hi])
+//    from a 256-entry row-pair table: one byte permute forms the address (the
+//    tables sit at a 64 KB-aligned shared address, so the byte drops straight
+//    into address bits 8..15) and one 32-bit load returns two weights. The
+//    four lanes that share a row pair read four bank copies, so every
+//    warp-wide lookup is conflict free whatever the indices are.
+//  * alpha/beta: one bf16x2 fma per pair, with per-pair (alpha_r, alpha_r+16)
+//    operands as stored, so w_hat is rounded once to bf16.
+//  * Operands: for M <= 8 the four looked-up pairs are used as they are, as
+//    one 16 x 16 tensor-core tile whose rows are the 16 row pairs; every token
+//    gets two output columns whose activation operand is zero in the slot of
+//    the other row of the pair, so the MMA itself separates the rows (no data
+//    movement). For M > 8 byte permutes turn the pairs into the usual two
+//    16-row tiles, which keeps one MMA per 8 tokens.
+//  * Work split: a thread block (one per SM) owns a contiguous range of
+//    (32-row panel, 64-column chunk) units (stream-K). For each panel its
+//    consumer warps build the 16 row-pair tables (64 KB) once, then split the
+//    panel's chunks. A producer warp streams every consumer warp's weights and
+//    alpha/beta, two chunks per bulk copy, into per-warp rings of full/empty
+//    mbarriers; the consumers load their activation columns straight from L2
+//    (two 128-bit loads per chunk, one chunk ahead). No block-wide barrier
+//    inside a panel. The warps' fp32 tiles are summed in warp order; a panel
+//    split between thread blocks is finished by the last one to arrive, which
+//    sums the partials in thread-block order (deterministic; nothing waits on
+//    another thread block).
 #include <cuda_bf16.h>
 
 #include <atomic>
@@ -44,11 +48,33 @@ namespace any4 {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kCtasPerSm = 2;
-constexpr int kMinAtomsPerCta = 16;
-constexpr uint32_t kTableBytes = 256 * 256;   // 256 entries x 64 words (2 tiles x 8 rows x 4 copies)
+constexpr int kMinUnitsPerCta = 32;
+constexpr int kPieceChunks = 2;                             // chunks per bulk copy
+constexpr int kSlotW = kPieceChunks * kChunkBytes;          // weights of one piece
+constexpr int kSlotBytes = kSlotW + kPieceChunks * kGroupScaleBytes;   // + up to 2 groups of alpha/beta
+constexpr int kMiscBytes = 1024;                            // mbarriers and flags
+constexpr uint32_t kTabAddr = 131072;        // shared-window address of the row-pair tables
+constexpr uint32_t kTabBytes = 65536;        // 256 entries x 2 halves x 8 pairs x 4 copies x 4 B
+constexpr uint32_t kRedAddr = kTabAddr + kTabBytes;
+constexpr long long kWaitLimitCycles = 4000000000ll;   // ~2 s: then the kernel records a timeout
+constexpr int kConsumerBar = 1;              // named barrier of the consumer warps
+
+// MODE 0: M <= 4, MODE 1: M <= 8 (row-pair operands, one or two column tiles
+// of 4 tokens); MODE 2: M <= 16 (row operands, two 8-token column tiles).
+template <int MODE>
+struct Cfg {
+  static constexpr bool kTr = MODE == 2;
+  static constexpr int kNt8 = MODE == 0 ? 1 : 2;                  // 8-column MMA tiles
+  static constexpr int kNW = MODE == 0 ? 16 : 8;                  // consumer warps
+  static constexpr int kThreads = (kNW + 2) * 32;                 // + producer and reducer warps
+  static constexpr int kNF = kTr ? 16 : 4 * kNt8;                 // fp32 results per lane
+  static constexpr int kNS = 3;                                   // ring depth (pieces)
+  static constexpr int kRingBytes = kNW * kNS * kSlotBytes;
+  static constexpr int kTileBytes = kNW * 32 * kNF * 4;           // the warps' fp32 tiles of a panel
+  static constexpr int kSmemBytes = (int)kRedAddr + 2 * kTileBytes;   // covers any window base
+  // everything below the tables, for a window that starts within 8 KB
+  static_assert(8192 + kMiscBytes + kRingBytes <= (int)kTabAddr, "rings overlap the tables");
+};
 
 struct Params {
   const uint16_t* x;
@@ -56,10 +82,11 @@ struct Params {
   uint16_t* y;
   float* partials;
   unsigned* counters;
+  unsigned* status;
   int m, n, k;
-  int katoms, groups, apg_shift;           // atoms per group = 1 << apg_shift
+  int kc, groups, g_shift;                  // chunks per panel, groups per row, log2(G)
   int ctas;
-  long long atoms;                          // blocks * katoms
+  long long units;
   size_t w_off, lut_off, ab_off;
 };
 
@@ -67,401 +94,449 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+__device__ __forceinline__ void consumer_sync(int threads) {
+  asm volatile("bar.sync %0, %1;" ::"n"(kConsumerBar), "r"(threads) : "memory");
+}
+
+// Named barriers: 1 = consumer warps; 2 + b = "warp tiles of buffer b
+// stored" (consumers arrive, the reducer waits); 4 + b = "buffer b read"
+// (the reducer arrives, the consumers wait before reusing it).
+__device__ __forceinline__ void named_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// Thread block whose unit range [floor(c*U/C), floor((c+1)*U/C)) holds unit u.
+__device__ __forceinline__ int cta_of_unit(long long u, long long U, int C) {
+  return (int)(((u + 1) * (long long)C - 1) / U);
 }
 
-// Thread block that owns atom a under the split a_begin(c) = floor(c * A / C).
-__device__ __forceinline__ int cta_of_atom(long long a, long long A, int C) {
-  return (int)(((a + 1) * (long long)C - 1) / A);
-}
-
-// Decode one packed word into the four bf16x2 operand registers of the
-// m16n8k16 tile (before alpha/beta). Row g (bits 0..15) from the register
-// planes, row g+8 (bytes 2 and 3) from the shared pair table.
-__device__ __forceinline__ void decode_word(uint32_t w, const uint32_t (&lo)[4],
-                                            const uint32_t (&hi)[4], uint32_t tab, uint32_t off,
-                                            uint32_t (&a)[4]) {
-  const uint32_t w7 = w & 0x7777u;                          // entry within a half table
-  const uint32_t sel = ((w >> 1) & 0x4444u) | 0x3210u;      // half 0 (byte j) or 1 (byte j+4)
-  const uint32_t pa = prmt(lo[0], lo[1], w7), pb = prmt(lo[2], lo[3], w7);
-  const uint32_t qa = prmt(hi[0], hi[1], w7), qb = prmt(hi[2], hi[3], w7);
-  const uint32_t l = prmt(pa, pb, sel), h = prmt(qa, qb, sel);
-  a[0] = prmt(l, h, 0x5140u);                               // tile columns 2t, 2t+1
-  a[2] = prmt(l, h, 0x7362u);                               // tile columns 2t+8, 2t+9
-  a[1] = lds32(tab + prmt(w, off, 0x5524u));                // entry = byte 2, times 256, + off
-  a[3] = lds32(tab + prmt(w, off, 0x5534u));                // entry = byte 3
-}
-
-template <int NT>
-__device__ __forceinline__ void store_y(const Params& p, int tile0, int lane,
-                                        const float (&v)[2][NT][4]) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int m = 8 * j + 2 * t + (i & 1);
-        const int n = (tile0 + tau) * kTileRows + g + 8 * (i >> 1);
-        if (m < p.m && n < p.n) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(v[tau][j][i]);
-          p.y[(size_t)m * p.n + n] = *reinterpret_cast<const uint16_t*>(&h);
-        }
-      }
-}
-
-// cp.async of 16 bytes global -> shared (no registers involved)
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-
-// The 32 rows x 16 LUT entries of one 32-row block (1 KB) into a shared slot.
-__device__ __forceinline__ void stage_lut(const Params& p, int block, uint32_t slot) {
-  if (threadIdx.x < 64)
-    cp_async16(slot + 16u * threadIdx.x,
-               p.packed + p.lut_off + (size_t)block * kBlockRows * 32 + 16u * threadIdx.x);
-  cp_async_commit();
-}
-
-template <int NT, int PF>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) linear_kernel(const Params p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const uint32_t tab = smem_u32(smem);
-  // warp partial tiles for the cross-warp sum; they reuse the table space,
-  // which is dead between the end of a block's streaming and the next build
-  float* red = reinterpret_cast<float*>(smem);
-  constexpr int kF = 2 * NT * 4;
-  const uint32_t lut_slot0 = tab + kTableBytes;   // 2 x 1 KB
-  const uint8_t* lut_smem = smem + kTableBytes;
-  // per-warp ring of PF atoms x 2 tiles x 512 bytes, filled by cp.async; each
-  // lane copies and later reads only its own 16 bytes per tile and atom
-  const uint32_t ring = lut_slot0 + 2048u + (uint32_t)(threadIdx.x >> 5) * (PF * 1024u) + 16u * (threadIdx.x & 31);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int KA = p.katoms, K = p.k;
-  const int apg = 1 << p.apg_shift;
-  const long long A = p.atoms;
-  const long long a_lo = (long long)blockIdx.x * A / p.ctas;
-  const long long a_hi = (long long)(blockIdx.x + 1) * A / p.ctas;
-  const int b_first = (int)(a_lo / KA);
-
-  // activation rows of this lane's B fragments: token 8j+g, columns
-  // 64*atom + 16*t .. +15 for the four steps of an atom. Tokens >= M repeat
-  // token M-1; their outputs are never stored.
-  const uint8_t* xrow[NT];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-    xrow[j] = reinterpret_cast<const uint8_t*>(p.x + (size_t)min(8 * j + g, p.m - 1) * K) + 32 * t;
-
-  // pair-table slice this thread builds: entry quarter, tile, row, bank copy
-  const int bq = threadIdx.x >> 6, btau = (threadIdx.x >> 5) & 1;
-  const int brow = (threadIdx.x >> 2) & 7, bcopy = threadIdx.x & 3;
-  const uint32_t build_addr = tab + (uint32_t)bq * 64u * 256u + 128u * btau + 16u * brow + 4u * bcopy;
-  // byte offset of this lane's bank copy inside an entry row, per tile
-  const uint32_t off[2] = {16u * g + 4u * t, 16u * g + 4u * t + 128u};
-
-  // ---- per-warp streaming state, primed one segment ahead
-  uint32_t xf[2][NT][4][2];
-  uint32_t sraw[4], snext[4];
-  auto seg_bounds = [&](long long sa, int& b, long long& se, int& wa0, int& wa1) {
-    b = (int)(sa / KA);
-    const long long bstart = (long long)b * KA;
-    se = min(a_hi, bstart + KA);
-    const int ka0 = (int)(sa - bstart), n_at = (int)(se - sa);
-    wa0 = ka0 + (int)((long long)warp * n_at / kWarps);
-    wa1 = ka0 + (int)((long long)(warp + 1) * n_at / kWarps);
-  };
-  auto wptr = [&](int b) {
-    return p.packed + p.w_off + (size_t)(2 * b) * KA * kAtomBytes + (size_t)lane * 16;
-  };
-  auto abptr = [&](int b) {
-    return reinterpret_cast<const uint32_t*>(p.packed + p.ab_off) +
-           (size_t)(2 * b) * p.groups * kTileRows + g;
-  };
-  auto load_x = [&](int atom, uint32_t (&dst)[NT][4][2]) {
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const uint8_t* src = xrow[j] + (size_t)atom * (kAtomK * 2);
-      const uint4 u0 = ld_nc_v4(src), u1 = ld_nc_v4(src + 16);
-      dst[j][0][0] = u0.x; dst[j][0][1] = u0.y; dst[j][1][0] = u0.z; dst[j][1][1] = u0.w;
-      dst[j][2][0] = u1.x; dst[j][2][1] = u1.y; dst[j][3][0] = u1.z; dst[j][3][1] = u1.w;
+// The chunks one consumer warp works on, in order: for every panel of the
+// thread block (units [u_lo, u_hi)), the warp's share [c, cend) of the
+// block's chunk range in that panel.
+template <int NW>
+struct ChunkCursor {
+  int panel, plast, c, cend;
+  long long u_lo, u_hi;
+  int kc, w;
+  __device__ void open() {
+    const long long pu = (long long)panel * kc;
+    const int a = (int)((u_lo > pu ? u_lo : pu) - pu);
+    const int b = (int)((u_hi < pu + kc ? u_hi : pu + kc) - pu);
+    c = a + (b - a) * w / NW;
+    cend = a + (b - a) * (w + 1) / NW;
+  }
+  __device__ void settle() {   // move past empty ranges
+    while (c >= cend && panel <= plast) {
+      ++panel;
+      if (panel <= plast) open();
     }
-  };
-  auto load_s = [&](const uint32_t* ab0, int atom, uint32_t (&dst)[4]) {
-    const uint32_t* ab1 = ab0 + (size_t)p.groups * kTileRows;
-    const size_t o = (size_t)(atom >> p.apg_shift) * kTileRows;
-    dst[0] = ld_nc_u32(ab0 + o); dst[1] = ld_nc_u32(ab0 + o + 8);
-    dst[2] = ld_nc_u32(ab1 + o); dst[3] = ld_nc_u32(ab1 + o + 8);
-  };
-  // weights of atom `atom` of block b into ring slot `slot` (one commit group,
-  // possibly empty, per call so that group counting stays uniform)
-  auto fetch = [&](int b, int atom, bool valid, int slot) {
-    if (valid) {
-      const uint8_t* w0 = wptr(b) + (size_t)atom * kAtomBytes;
-      cp_async16(ring + (uint32_t)slot * 1024u, w0);
-      cp_async16(ring + (uint32_t)slot * 1024u + 512u, w0 + (size_t)KA * kAtomBytes);
+  }
+  __device__ void start(int p0, int p1, long long lo, long long hi, int kc_, int w_) {
+    panel = p0; plast = p1; u_lo = lo; u_hi = hi; kc = kc_; w = w_;
+    open();
+    settle();
+  }
+  __device__ bool valid() const { return panel <= plast; }
+};
+
+// Waits for phase `parity` of mbarrier `bar`, at most ~kWaitLimitCycles; after
+// a timeout (or one seen earlier by this block) it returns without waiting.
+__device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile uint32_t* abort) {
+  if (mbar_try_wait(bar, parity)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      *abort = 1u;
+      return;
     }
-    cp_async_commit();
-  };
-  // first loads of a warp's range: weights of the first PF atoms, activations
-  // and scales of the first atom
-  auto prime = [&](int b, int wa0, int wa1, bool with_x) {
-#pragma unroll
-    for (int j = 0; j < PF; ++j) fetch(b, wa0 + j, wa0 + j < wa1, j);
-    if (wa0 >= wa1) return;
-    if (with_x) load_x(wa0, xf[0]);
-    load_s(abptr(b), wa0, sraw);
+  }
+}
+
+// (token, row within the panel) of result i of lane `ln`.
+template <int MODE>
+__device__ __forceinline__ void out_pos(int ln, int i, int& token, int& row) {
+  const int g = ln >> 2, t = ln & 3;
+  if (!Cfg<MODE>::kTr) {
+    const int h = i >> 2, q = i & 3;      // D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]
+    token = 4 * h + t;
+    row = g + (q == 1 ? 16 : q == 2 ? 8 : q == 3 ? 24 : 0);
+  } else {
+    const int tile = i >> 3, h = (i >> 2) & 1, q = i & 3;
+    token = 8 * h + 2 * t + (q & 1);
+    row = 16 * tile + g + 8 * (q >> 1);
+  }
+}
+
+template <int MODE>
+__device__ __forceinline__ void store_out(const Params& p, int P, int o, float v) {
+  constexpr int NF = Cfg<MODE>::kNF;
+  int token, row;
+  out_pos<MODE>(o / NF, o % NF, token, row);
+  const int n = P * kPanelRows + row;
+  if (token < p.m && n < p.n) {
+    const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+    p.y[(size_t)token * p.n + n] = *reinterpret_cast<const uint16_t*>(&hv);
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Params p) {
+  using C = Cfg<MODE>;
+  constexpr int NS = C::kNS, NF = C::kNF, NW = C::kNW, NCT = NW * 32;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // Shared window: [mbarriers, flags][per-warp rings] ... [row-pair tables at
+  // kTabAddr][two buffers of warp tiles]. The dynamic window starts at a small
+  // fixed offset, so the rings fit below the tables; if they ever do not,
+  // record it and leave before touching anything else.
+  const uint32_t ring0 = base + kMiscBytes;
+  if (ring0 + (uint32_t)C::kRingBytes > kTabAddr) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tid == 0) atomicOr(p.status, 2u);
+    return;
+  }
+  volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + 1016);
+  auto full_bar = [&](int w, int s) { return base + (uint32_t)(w * NS + s) * 16u; };
+  auto empty_bar = [&](int w, int s) { return base + (uint32_t)(w * NS + s) * 16u + 8u; };
+  auto slot_addr = [&](int w, int s) { return ring0 + (uint32_t)(w * NS + s) * kSlotBytes; };
+  float* tiles = reinterpret_cast<float*>(smem + (kRedAddr - base));   // [2][NW][32][NF]
+
+  const long long U = p.units;
+  const int kc = p.kc;
+  const long long u_lo = (long long)blockIdx.x * U / p.ctas;
+  const long long u_hi = (long long)(blockIdx.x + 1) * U / p.ctas;
+  const int P0 = (int)(u_lo / kc), P1 = (int)((u_hi - 1) / kc);
+  auto is_split = [&](int P) {
+    const long long pu = (long long)P * kc;
+    return !(pu >= u_lo && pu + kc <= u_hi);
   };
 
-  long long sa = a_lo;
-  int b, wa0, wa1;
-  long long se;
-  seg_bounds(sa, b, se, wa0, wa1);
-  // Only the packed weight (immutable) is read before the grid dependency
-  // resolves, so with programmatic dependent launch this prologue overlaps the
-  // previous kernel on the stream; activations, y and the workspace are
-  // touched only after griddepcontrol.wait.
-  prime(b, wa0, wa1, false);
-  uint32_t lut_cur = lut_slot0;
-  stage_lut(p, b, lut_cur);
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  cp_async_wait_all();
+  if (tid == 0) *abort = 0u;
+  if (tid < NW * NS) {
+    mbar_init(full_bar(tid / NS, tid % NS), 1);
+    mbar_init(empty_bar(tid / NS, tid % NS), 32);
+  }
+  fence_mbar_init();
   __syncthreads();
-  bool first_seg = true;
-  int split0 = -1, split1 = -1;   // split blocks whose partials await the final count
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  while (true) {
-    const int tile0 = 2 * b;
-    const uint8_t* lut_here = lut_smem + (lut_cur - lut_slot0);
-    {
-      // pair tables of rows 8..15 of both tiles: entry e = (LUT[e & 15], LUT[e >> 4])
-      const uint4* src = reinterpret_cast<const uint4*>(lut_here + (16 * btau + 8 + brow) * 32);
-      const uint4 u0 = src[0], u1 = src[1];
-      const uint32_t L[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-      // high nibbles of this quarter are 4*bq .. 4*bq+3, i.e. pairs L[2bq], L[2bq+1]
-      const uint32_t h0 = bq == 0 ? u0.x : bq == 1 ? u0.z : bq == 2 ? u1.x : u1.z;
-      const uint32_t h1 = bq == 0 ? u0.y : bq == 1 ? u0.w : bq == 2 ? u1.y : u1.w;
-#pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const uint32_t sel = ((j & 1) ? 0x32u : 0x10u) | ((((j >> 4) & 1) ? 0x76u : 0x54u) << 8);
-        sts32(build_addr + (uint32_t)j * 256u, prmt(L[(j & 15) >> 1], (j >> 5) ? h1 : h0, sel));
-      }
+  // =========================== producer warp ===============================
+  // Lane w < NW streams consumer warp w's pieces (up to two chunks of one
+  // panel) in the order the warp uses them. It reads only the packed weight,
+  // which is immutable, so it needs no grid-dependency wait: with
+  // programmatic dependent launch it runs ahead while the previous kernel on
+  // the stream finishes.
+  if (warp == NW) {
+    ChunkCursor<NW> cur;
+    cur.start(P0, P1, u_lo, u_hi, kc, lane);
+    if (lane >= NW) cur.panel = P1 + 1;   // lanes without a consumer warp
+    const uint8_t* wbase = p.packed + p.w_off;
+    const uint8_t* abase = p.packed + p.ab_off;
+    int issued = 0;   // pieces issued so far; piece q uses slot q % NS for the (q / NS)-th time
+    while (cur.valid()) {
+      const int slot = issued % NS;
+      const int n = min(kPieceChunks, cur.cend - cur.c);
+      const int g_lo = (cur.c * kChunkCols) >> p.g_shift;
+      const int g_hi = ((cur.c + n) * kChunkCols - 1) >> p.g_shift;
+      const uint32_t wbytes = (uint32_t)n * kChunkBytes;
+      const uint32_t sbytes = (uint32_t)(g_hi - g_lo + 1) * kGroupScaleBytes;
+      if (issued >= NS)   // the consumer's release of the slot's previous use
+        wait_bar(empty_bar(lane, slot), (uint32_t)(issued / NS - 1) & 1u, abort);
+      if (*abort) break;
+      const uint32_t fb = full_bar(lane, slot), dst = slot_addr(lane, slot);
+      mbar_arrive_expect_tx(fb, wbytes + sbytes);
+      bulk_g2s(dst, wbase + (((size_t)cur.panel * kc + cur.c) << 10), wbytes, fb);
+      bulk_g2s(dst + kSlotW, abase + (((size_t)cur.panel * p.groups + g_lo) << 7), sbytes, fb);
+      ++issued;
+      cur.c += n;
+      cur.settle();
     }
-    // this lane's row-g tables of both tiles as low-byte / high-byte planes
-    uint32_t lo[2][4], hi[2][4];
-#pragma unroll
-    for (int tau = 0; tau < 2; ++tau) {
-      const uint4* src = reinterpret_cast<const uint4*>(lut_here + (16 * tau + g) * 32);
-      const uint4 u0 = src[0], u1 = src[1];
-      const uint32_t L[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo[tau][i] = prmt(L[2 * i], L[2 * i + 1], 0x6420u);
-        hi[tau][i] = prmt(L[2 * i], L[2 * i + 1], 0x7531u);
-      }
-    }
-    // next segment (if any): its LUT rows start moving now
-    const bool has_next = se < a_hi;
-    int nb = 0, nwa0 = 0, nwa1 = 0;
-    long long nse = 0;
-    if (has_next) {
-      seg_bounds(se, nb, nse, nwa0, nwa1);
-      lut_cur = lut_slot0 + (lut_cur == lut_slot0 ? 1024u : 0u);
-      stage_lut(p, nb, lut_cur);
-    }
-    __syncthreads();   // tables ready
-    if (first_seg) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      if (wa0 < wa1) load_x(wa0, xf[0]);
-      first_seg = false;
-    }
+    return;
+  }
 
-    float acc[2][NT][4];
+  // =========================== reducer warp ================================
+  // Sums the consumer warps' fp32 tiles of each panel in warp order (a fixed
+  // tree) and writes y. A panel split between thread blocks (stream-K) is
+  // finished by the block that holds the panel's first unit; it processes
+  // the panel last, while the other contributors process it first and
+  // publish their partial sum at once (release-increment of the panel's
+  // counter). The finisher collects their partials while its consumers still
+  // work on the panel, adds them after its own sum in thread-block order
+  // (deterministic) and resets the counter for the next call.
+  if (warp == NW + 1) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // y, partials, counters
+    for (int P = P0; P <= P1; ++P) {
+      const int b = (P - P0) & 1;
+      const bool split = is_split(P);
+      const long long pu = (long long)P * kc;
+      const bool finisher = split && pu >= u_lo;
+      const int c_first = split ? cta_of_unit(pu, U, p.ctas) : 0;
+      const int c_last = split ? cta_of_unit(pu + kc - 1, U, p.ctas) : 0;
+      float other[NF];
 #pragma unroll
-    for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[tau][j][i] = 0.0f;
-
-    if (wa0 < wa1) {
-      const uint32_t* ab0 = abptr(b);
-      uint32_t al[4], be[4];   // (alpha, alpha), (beta, beta): rows g, g+8 of both tiles
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { al[i] = prmt(sraw[i], sraw[i], 0x1010u); be[i] = prmt(sraw[i], sraw[i], 0x3232u); }
-      if (wa0 + 1 < wa1 && ((wa0 + 1) & (apg - 1)) == 0) load_s(ab0, wa0 + 1, snext);
-
-      for (int a0 = wa0; a0 < wa1; a0 += PF) {
-#pragma unroll
-        for (int jj = 0; jj < PF; ++jj) {
-          const int a = a0 + jj;
-          if (a >= wa1) break;
-          cp_async_wait<PF - 1>();                      // this atom's weights have landed
-          const uint4 v0 = lds128(ring + (uint32_t)jj * 1024u);
-          const uint4 v1 = lds128(ring + (uint32_t)jj * 1024u + 512u);
-          fetch(b, a + PF, a + PF < wa1, jj);
-          uint32_t (&xc)[NT][4][2] = xf[jj & 1];
-          if (a + 1 < wa1) load_x(a + 1, xf[(jj + 1) & 1]);
-          if (a != wa0 && (a & (apg - 1)) == 0) {          // first atom of a new group
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              al[i] = prmt(snext[i], snext[i], 0x1010u);
-              be[i] = prmt(snext[i], snext[i], 0x3232u);
-            }
+      for (int i = 0; i < NF; ++i) other[i] = 0.0f;
+      if (finisher && c_last > c_first) {
+        const unsigned need = (unsigned)(c_last - c_first);
+        if (lane == 0 && ld_acquire(p.counters + P) < need) {
+          const long long t0 = clock64();
+          while (ld_acquire(p.counters + P) < need) {
+            if (*abort) break;
+            if (clock64() - t0 > kWaitLimitCycles) { *abort = 1u; break; }
           }
-          if (a + 1 < wa1 && ((a + 1) & (apg - 1)) == 0) load_s(ab0, a + 1, snext);
-          const uint32_t words[2][4] = {{v0.x, v0.y, v0.z, v0.w}, {v1.x, v1.y, v1.z, v1.w}};
+        }
+        __syncwarp();
+        (void)ld_acquire(p.counters + P);   // this lane's acquire of the publishers' stores
+        for (int c = c_first + 1; c <= c_last; ++c) {
+          const float* src = p.partials + ((size_t)c * 32 + lane) * NF;
 #pragma unroll
-          for (int s = 0; s < 4; ++s)
-#pragma unroll
-            for (int tau = 0; tau < 2; ++tau) {
-              uint32_t af[4];
-              decode_word(words[tau][s], lo[tau], hi[tau], tab, off[tau], af);
-              af[0] = fma_bf16x2(af[0], al[2 * tau], be[2 * tau]);
-              af[2] = fma_bf16x2(af[2], al[2 * tau], be[2 * tau]);
-              af[1] = fma_bf16x2(af[1], al[2 * tau + 1], be[2 * tau + 1]);
-              af[3] = fma_bf16x2(af[3], al[2 * tau + 1], be[2 * tau + 1]);
-#pragma unroll
-              for (int j = 0; j < NT; ++j) mma_m16n8k16(acc[tau][j], af, xc[j][s][0], xc[j][s][1]);
-            }
+          for (int i = 0; i < NF; ++i) other[i] += __ldcg(src + i);
         }
       }
-    }
-    // the next segment's first loads leave before this one's reduction
-    if (has_next) prime(nb, nwa0, nwa1, true);
-
-    // ---- sum the warps' tiles in warp order (the table space is free once
-    // every warp is past its lookups)
-    __syncthreads();
-    {
-      float4* dst = reinterpret_cast<float4*>(red + ((size_t)warp * 32 + lane) * kF);
+      named_sync(2 + b, NCT + 32);   // tiles of panel P stored
+      const float* tb = tiles + (size_t)b * NW * 32 * NF + (size_t)lane * NF;
+      float v[NF];
 #pragma unroll
-      for (int tau = 0; tau < 2; ++tau)
+      for (int i = 0; i < NF; ++i) {
+        float t[NW];
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-          dst[tau * NT + j] = make_float4(acc[tau][j][0], acc[tau][j][1], acc[tau][j][2], acc[tau][j][3]);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      const long long bstart = (long long)b * KA;
-      float v[2][NT][4];
+        for (int w = 0; w < NW; ++w) t[w] = tb[(size_t)w * 32 * NF + i];
 #pragma unroll
-      for (int tau = 0; tau < 2; ++tau)
+        for (int span = 1; span < NW; span *= 2)
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) v[tau][j][i] = 0.0f;
-      for (int w = 0; w < kWarps; ++w) {
-        const float4* src = reinterpret_cast<const float4*>(red + ((size_t)w * 32 + lane) * kF);
-#pragma unroll
-        for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            const float4 f = src[tau * NT + j];
-            v[tau][j][0] += f.x; v[tau][j][1] += f.y; v[tau][j][2] += f.z; v[tau][j][3] += f.w;
-          }
+          for (int w = 0; w + span < NW; w += 2 * span) t[w] += t[w + span];
+        v[i] = t[0];
       }
-      if (sa == bstart && se == bstart + KA) {
-        store_y<NT>(p, tile0, lane, v);                       // the whole block is ours
+      if (P + 2 <= P1) named_arrive(4 + b, NCT + 32);   // buffer b may be reused
+      if (!split || finisher) {
+#pragma unroll
+        for (int i = 0; i < NF; ++i) store_out<MODE>(p, P, lane * NF + i, v[i] + other[i]);
+        if (split && lane == 0) p.counters[P] = 0u;   // ready for the next call
       } else {
-        // split block: store the fp32 partial now; the arrival count (and the
-        // sum, if this thread block turns out to be the last) waits for the end
-        // of the thread block, off the streaming path
-        const int my_slot = 2 * blockIdx.x + (b == b_first ? 0 : 1);
-        float4* dst = reinterpret_cast<float4*>(p.partials + ((size_t)my_slot * 32 + lane) * kF);
+        float* dst = p.partials + ((size_t)blockIdx.x * 32 + lane) * NF;
 #pragma unroll
-        for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-          for (int j = 0; j < NT; ++j)
-            __stcg(dst + tau * NT + j, make_float4(v[tau][j][0], v[tau][j][1], v[tau][j][2], v[tau][j][3]));
-        if (b == b_first) split0 = b; else split1 = b;
+        for (int i = 0; i < NF; ++i) __stcg(dst + i, v[i]);
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) red_release_add(p.counters + P, 1u);
       }
     }
-    if (!has_next) break;
-    cp_async_wait<PF>();   // the LUT rows (older than the PF weight groups of prime)
-    __syncthreads();       // reduction reads done, next LUT rows visible
-    sa = se;
-    b = nb; se = nse; wa0 = nwa0; wa1 = nwa1;
+    if (lane == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
+    return;
   }
 
-  // ---- arrival counts of the split blocks; the last thread block of a block
-  // sums all partials in thread-block order and writes y
-  if (warp == 0 && (split0 >= 0 || split1 >= 0)) {
-    __threadfence();   // this warp's partial stores before the counts
-    __syncwarp();
-    for (int q = 0; q < 2; ++q) {
-      const int sb = q == 0 ? split0 : split1;
-      if (sb < 0) continue;
-      unsigned prev = 0;
-      if (lane == 0) prev = atomicAdd(p.counters + sb, 1u);
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      const long long bstart = (long long)sb * KA;
-      const int c_first = cta_of_atom(bstart, A, p.ctas);
-      const int c_last = cta_of_atom(bstart + KA - 1, A, p.ctas);
-      if (prev != (unsigned)(c_last - c_first)) continue;
-      __threadfence();
-      float sum[2][NT][4];
+  // =========================== consumer warps ==============================
+  const int g = lane >> 2, t = lane & 3;
+
+  // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
+  // 8*blh .. 8*blh+7; every entry goes to its four bank copies
+  constexpr int kBuildPer = 512 / NCT;
+  const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off);
+  // this thread's LUT values of the panel being built (lw/lh) and of the
+  // next one (nw/nh), loaded a full panel ahead
+  uint4 lw[kBuildPer], nw[kBuildPer];
+  uint32_t lh[kBuildPer], nh[kBuildPer];
+  auto load_lut = [&](int P, uint4 (&dw)[kBuildPer], uint32_t (&dh)[kBuildPer]) {
 #pragma unroll
-      for (int tau = 0; tau < 2; ++tau)
+    for (int r = 0; r < kBuildPer; ++r) {
+      const int task = tid + r * NCT;
+      const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
+      const int br0 = (brp & 7) + 8 * (brp >> 3);
+      dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
+      dh[r] = ld_nc_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+    }
+  };
+  load_lut(P0, lw, lh);
+  if (P0 < P1) load_lut(P0 + 1, nw, nh);
+
+  // lookup address bases: byte b of a word goes to address bits 8..15
+  const uint32_t baseA = kTabAddr | ((uint32_t)g << 4) | ((uint32_t)t << 2);   // pairs (g, g+16)
+  const uint32_t baseB = baseA | 128u;                                         // pairs (g+8, g+24)
+
+  // Activation operands. Tile h serves tokens 4h.. (row-pair mode: lane g
+  // feeds output column g = 2j + p of token j, zero in the slot of the other
+  // row of the pair) or 8h.. (row mode: lane g feeds token 8h+g). A lane whose
+  // token is >= M reads token 0 (a cached line) and zeroes its operand.
+  constexpr int NX = C::kTr ? 2 : C::kNt8;
+  const uint16_t* xrow[NX];
+  uint32_t selb0[NX], selb1[NX], xmask[NX];
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
+  for (int h = 0; h < NX; ++h) {
+    const int j = C::kTr ? 8 * h + g : 4 * h + (g >> 1);
+    const bool ok = j < p.m;
+    xrow[h] = p.x + (size_t)(ok ? j : 0) * p.k + 16 * t;
+    selb0[h] = !ok ? 0x4444u : (g & 1) ? 0x1044u : 0x4410u;
+    selb1[h] = !ok ? 0x4444u : (g & 1) ? 0x3244u : 0x4432u;
+    xmask[h] = ok ? 0xffffffffu : 0u;
+  }
+  // words s = 0..7 of a chunk: columns 16t + 2s, +1 of the chunk
+  uint4 xn[NX][2];
+  auto load_x = [&](int c) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sum[tau][j][i] = 0.0f;
-      constexpr int kBatch = 4;
-      for (int c0 = c_first; c0 <= c_last; c0 += kBatch) {
-        float4 f[kBatch][2 * NT];
+    for (int h = 0; h < NX; ++h) {
+      xn[h][0] = ld_nc_v4(xrow[h] + (size_t)c * kChunkCols);
+      xn[h][1] = ld_nc_v4(xrow[h] + (size_t)c * kChunkCols + 8);
+    }
+  };
+  ChunkCursor<NW> xc;   // the chunk whose activations load next
+  xc.start(P0, P1, u_lo, u_hi, kc, warp);
+
+  int q = 0;   // pieces consumed; piece q sits in slot q % NS, phase (q / NS) & 1
+
+  for (int P = P0; P <= P1; ++P) {
+    // ---- build the 16 row-pair tables of panel P
 #pragma unroll
-        for (int qq = 0; qq < kBatch; ++qq) {
-          const int c = c0 + qq;
-          if (c <= c_last) {
-            const long long cb = (long long)c * A / p.ctas;
-            const int slot = 2 * c + ((long long)sb == cb / KA ? 0 : 1);
-            const float4* src = reinterpret_cast<const float4*>(p.partials + ((size_t)slot * 32 + lane) * kF);
+    for (int r = 0; r < kBuildPer; ++r) {
+      const int task = tid + r * NCT;
+      const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
+      const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
+      const uint32_t L[4] = {lw[r].x, lw[r].y, lw[r].z, lw[r].w};
 #pragma unroll
-            for (int u = 0; u < 2 * NT; ++u) f[qq][u] = __ldcg(src + u);
-          } else {
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t e = (uint32_t)(8 * blh + i) | ((uint32_t)bhi << 4);
+        const uint32_t v = prmt(L[i >> 1], lh[r], (i & 1) ? 0x5432u : 0x5410u);
+        sts128(bdst + (e << 8), v, v, v, v);
+      }
+    }
 #pragma unroll
-            for (int u = 0; u < 2 * NT; ++u) f[qq][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < kBuildPer; ++r) { lw[r] = nw[r]; lh[r] = nh[r]; }
+    if (P + 1 < P1) load_lut(P + 2, nw, nh);
+    if (P == P0) {
+      // activations, y and the workspace are touched only from here on
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (xc.valid()) {
+        load_x(xc.c);
+        ++xc.c;
+        xc.settle();
+      }
+    }
+    consumer_sync(NCT);   // tables ready
+
+    float acc[NF];
+#pragma unroll
+    for (int i = 0; i < NF; ++i) acc[i] = 0.0f;
+
+    ChunkCursor<NW> mine;
+    mine.panel = P; mine.plast = P1; mine.u_lo = u_lo; mine.u_hi = u_hi; mine.kc = kc; mine.w = warp;
+    mine.open();
+    for (int pc = mine.c; pc < mine.cend; pc += kPieceChunks) {
+      const int n = min(kPieceChunks, mine.cend - pc);
+      const int g_lo = (pc * kChunkCols) >> p.g_shift;
+      const int slot = q % NS;
+      const uint32_t sb = slot_addr(warp, slot);
+      wait_bar(full_bar(warp, slot), (uint32_t)(q / NS) & 1u, abort);
+      for (int cc = 0; cc < n; ++cc) {
+        const int c = pc + cc;
+        uint4 xv[NX][2];
+#pragma unroll
+        for (int h = 0; h < NX; ++h) { xv[h][0] = xn[h][0]; xv[h][1] = xn[h][1]; }
+        if (xc.valid()) {   // next chunk's activations, one chunk ahead
+          load_x(xc.c);
+          ++xc.c;
+          xc.settle();
+        }
+        const uint32_t wsb = sb + (uint32_t)cc * kChunkBytes;
+        const uint4 wa = lds128(wsb + 16u * lane), wb = lds128(wsb + 512u + 16u * lane);
+        // alpha/beta pairs of (g, g+16) and (g+8, g+24) for this chunk's group
+        const uint4 sc = lds128(sb + kSlotW + ((uint32_t)(((c * kChunkCols) >> p.g_shift) - g_lo) << 7) +
+                                16u * g);
+        // release the slot once its last loads have landed (acc[0] depends on
+        // every load of the piece's earlier chunk)
+        if (cc == n - 1) mbar_arrive_after(empty_bar(warp, slot), wa.x, wb.x, sc.x, __float_as_uint(acc[0]));
+        const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        uint32_t xw[NX][8];
+#pragma unroll
+        for (int h = 0; h < NX; ++h) {
+          xw[h][0] = xv[h][0].x; xw[h][1] = xv[h][0].y; xw[h][2] = xv[h][0].z; xw[h][3] = xv[h][0].w;
+          xw[h][4] = xv[h][1].x; xw[h][5] = xv[h][1].y; xw[h][6] = xv[h][1].z; xw[h][7] = xv[h][1].w;
+        }
+        if (!C::kTr) {
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            uint32_t a[4];
+            a[0] = lds32(prmt(w[s], baseA, 0x7604u));
+            a[1] = lds32(prmt(w[s], baseB, 0x7614u));
+            a[2] = lds32(prmt(w[s], baseA, 0x7624u));
+            a[3] = lds32(prmt(w[s], baseB, 0x7634u));
+            a[0] = fma_bf16x2(a[0], sc.x, sc.y);
+            a[2] = fma_bf16x2(a[2], sc.x, sc.y);
+            a[1] = fma_bf16x2(a[1], sc.z, sc.w);
+            a[3] = fma_bf16x2(a[3], sc.z, sc.w);
+#pragma unroll
+            for (int h = 0; h < NX; ++h) {
+              float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[4 * h]);
+              mma_m16n8k16(d, a, prmt(xw[h][s], 0u, selb0[h]), prmt(xw[h][s], 0u, selb1[h]));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < NX; ++h)
+#pragma unroll
+            for (int s = 0; s < 8; ++s) xw[h][s] &= xmask[h];
+#pragma unroll
+          for (int s = 0; s < 8; s += 2) {
+            uint32_t e[2][4];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              e[u][0] = lds32(prmt(w[s + u], baseA, 0x7604u));
+              e[u][1] = lds32(prmt(w[s + u], baseB, 0x7614u));
+              e[u][2] = lds32(prmt(w[s + u], baseA, 0x7624u));
+              e[u][3] = lds32(prmt(w[s + u], baseB, 0x7634u));
+              e[u][0] = fma_bf16x2(e[u][0], sc.x, sc.y);
+              e[u][2] = fma_bf16x2(e[u][2], sc.x, sc.y);
+              e[u][1] = fma_bf16x2(e[u][1], sc.z, sc.w);
+              e[u][3] = fma_bf16x2(e[u][3], sc.z, sc.w);
+            }
+#pragma unroll
+            for (int tile = 0; tile < 2; ++tile) {
+              const uint32_t sel = tile ? 0x7632u : 0x5410u;
+              const uint32_t a[4] = {prmt(e[0][0], e[0][2], sel), prmt(e[0][1], e[0][3], sel),
+                                     prmt(e[1][0], e[1][2], sel), prmt(e[1][1], e[1][3], sel)};
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[8 * tile + 4 * h]);
+                mma_m16n8k16(d, a, xw[h][s], xw[h][s + 1]);
+              }
+            }
           }
         }
-#pragma unroll
-        for (int qq = 0; qq < kBatch; ++qq)
-#pragma unroll
-          for (int tau = 0; tau < 2; ++tau)
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-              const float4 u = f[qq][tau * NT + j];
-              sum[tau][j][0] += u.x; sum[tau][j][1] += u.y; sum[tau][j][2] += u.z; sum[tau][j][3] += u.w;
-            }
       }
-      store_y<NT>(p, 2 * sb, lane, sum);
-      if (lane == 0) p.counters[sb] = 0u;   // ready for the next call
+      ++q;
     }
+
+    // ---- hand the warp tiles to the reducer warp (double-buffered)
+    const int b = (P - P0) & 1;
+    if (P - P0 >= 2) named_sync(4 + b, NCT + 32);   // the reducer is done with buffer b
+    {
+      float4* dst = reinterpret_cast<float4*>(tiles + (size_t)b * NW * 32 * NF + (size_t)(warp * 32 + lane) * NF);
+#pragma unroll
+      for (int i = 0; i < NF / 4; ++i)
+        dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+    }
+    named_arrive(2 + b, NCT + 32);
+    consumer_sync(NCT);   // every consumer is past its lookups: the tables are free
   }
+  if (tid == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
 }
 
-constexpr int kRing = 4;   // atoms in flight per warp through the shared-memory ring
-
-size_t smem_bytes(int nt) {
-  (void)nt;   // the cross-warp sum reuses the table space
-  return kTableBytes + 2 * 1024 + (size_t)kWarps * kRing * 1024;
+template <int MODE>
+cudaError_t allow_smem_mode() {
+  return cudaFuncSetAttribute(linear_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<MODE>::kSmemBytes);
 }
 
 cudaError_t allow_large_smem() {
@@ -471,25 +546,42 @@ cudaError_t allow_large_smem() {
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (done_mask.load(std::memory_order_relaxed) & bit) return cudaSuccess;
-  e = cudaFuncSetAttribute(linear_kernel<1, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(1));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(linear_kernel<2, kRing>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(2));
+  e = allow_smem_mode<0>();
+  if (e == cudaSuccess) e = allow_smem_mode<1>();
+  if (e == cudaSuccess) e = allow_smem_mode<2>();
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_relaxed);
   return e;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t stream) {
+  // programmatic dependent launch: this kernel's weight prologue may overlap the
+  // tail of the previous kernel on the stream (see griddepcontrol in the kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.ctas);
+  cfg.blockDim = dim3(Cfg<MODE>::kThreads);
+  cfg.dynamicSmemBytes = Cfg<MODE>::kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, linear_kernel<MODE>, p);
 }
 
 }  // namespace
 
 LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   LinearPlan pl{};
-  pl.nt = m > 8 ? 2 : 1;
-  pl.atoms = (long long)(L.tiles / 2) * L.katoms;
-  long long c = pl.atoms / kMinAtomsPerCta;
-  const long long cap = (long long)num_sms * kCtasPerSm;
-  if (c > cap) c = cap;
+  pl.mode = m <= 4 ? 0 : m <= 8 ? 1 : 2;
+  pl.nf = pl.mode == 0 ? 4 : pl.mode == 1 ? 8 : 16;
+  pl.units = (long long)L.panels * L.kchunks;
+  long long c = pl.units / kMinUnitsPerCta;
+  if (c > num_sms) c = num_sms;
   if (c < 1) c = 1;
   pl.ctas = (int)c;
-  pl.partials_bytes = (size_t)2 * pl.ctas * 32 * (2 * pl.nt * 4) * sizeof(float);
+  pl.partials_bytes = (size_t)pl.ctas * 32 * pl.nf * sizeof(float);
   pl.workspace_bytes = kHeaderBytes + pl.partials_bytes;
   return pl;
 }
@@ -505,28 +597,20 @@ cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout
   p.y = y;
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   p.counters = reinterpret_cast<unsigned*>(ws);
+  p.status = reinterpret_cast<unsigned*>(ws + kCountersBytes);
   p.partials = reinterpret_cast<float*>(ws + kHeaderBytes);
   p.m = m; p.n = L.n; p.k = L.k;
-  p.katoms = L.katoms; p.groups = L.groups;
-  p.apg_shift = 0;
-  while ((kAtomK << p.apg_shift) < L.g) ++p.apg_shift;
+  p.kc = L.kchunks; p.groups = L.groups;
+  p.g_shift = 0;
+  while ((1 << p.g_shift) < L.g) ++p.g_shift;
   p.ctas = plan.ctas;
-  p.atoms = plan.atoms;
+  p.units = plan.units;
   p.w_off = L.w_off; p.lut_off = L.lut_off; p.ab_off = L.ab_off;
-  // programmatic dependent launch: this kernel's weight prologue may overlap the
-  // tail of the previous kernel on the stream (see griddepcontrol in the kernel)
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.ctas);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem_bytes(plan.nt);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (plan.nt == 1) return cudaLaunchKernelEx(&cfg, linear_kernel<1, kRing>, p);
-  return cudaLaunchKernelEx(&cfg, linear_kernel<2, kRing>, p);
+  switch (plan.mode) {
+    case 0: return launch_mode<0>(p, plan, stream);
+    case 1: return launch_mode<1>(p, plan, stream);
+    default: return launch_mode<2>(p, plan, stream);
+  }
 }
 
 }  // namespace any4

@@ -13,6 +13,31 @@
 
 namespace any4 {
 
+// Word e of the weight section: e = ((panel*kchunks + chunk)*2 + h)*128 + lane*4 + i,
+// step s = 4*h + i of the chunk, lane = 4*g + t, columns c0 = 64*chunk + 16t + 2s
+// and c0 + 1.
+struct WordPos {
+  size_t panel;
+  int g, t, c0;
+};
+
+__device__ __forceinline__ WordPos word_pos(size_t e, int kchunks) {
+  WordPos q;
+  const int i = (int)(e & 3);
+  const int lane = (int)((e >> 2) & 31);
+  const int h = (int)((e >> 7) & 1);
+  const size_t pc = e >> 8;
+  const int chunk = (int)(pc % kchunks);
+  q.panel = pc / kchunks;
+  q.g = lane >> 2;
+  q.t = lane & 3;
+  q.c0 = chunk * kChunkCols + 16 * q.t + 2 * (4 * h + i);
+  return q;
+}
+
+// Byte b of a word: rows (r, r+16) with r = g + 8*(b & 1), column c0 + (b >> 1).
+__device__ __forceinline__ int byte_row(int g, int b) { return g + 8 * (b & 1); }
+
 // One thread per packed 32-bit word.
 __global__ void pack_weights_kernel(const uint8_t* __restrict__ idx_nib, Layout L,
                                     uint32_t* __restrict__ out) {
@@ -20,21 +45,17 @@ __global__ void pack_weights_kernel(const uint8_t* __restrict__ idx_nib, Layout 
   const size_t row_bytes = (size_t)L.k / 2;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
-    const int step = (int)(e & 3);
-    const int lane = (int)((e >> 2) & 31);
-    const size_t tile_atom = e >> 7;
-    const int atom = (int)(tile_atom % L.katoms);
-    const size_t tile = tile_atom / L.katoms;
-    const int g = lane >> 2, t = lane & 3;
-    const size_t row0 = tile * kTileRows + g, row1 = row0 + 8;
-    const size_t j0 = (size_t)atom * (kAtomK / 2) + t * 8 + step * 2;   // column 64a+16t+4s
-    const size_t j1 = j0 + 1;                                            // column +2
+    const WordPos q = word_pos(e, L.kchunks);
     uint32_t v = 0;
-    if (row0 < (size_t)L.n)
-      v |= (uint32_t)idx_nib[row0 * row_bytes + j0] | ((uint32_t)idx_nib[row0 * row_bytes + j1] << 8);
-    if (row1 < (size_t)L.n)
-      v |= ((uint32_t)idx_nib[row1 * row_bytes + j0] << 16) |
-           ((uint32_t)idx_nib[row1 * row_bytes + j1] << 24);
+    for (int b = 0; b < 4; ++b) {
+      const int col = q.c0 + (b >> 1);
+      for (int u = 0; u < 2; ++u) {
+        const size_t row = q.panel * kPanelRows + byte_row(q.g, b) + 16 * u;
+        if (row >= (size_t)L.n) continue;
+        const uint32_t nib = (idx_nib[row * row_bytes + col / 2] >> (4 * (col & 1))) & 0xFu;
+        v |= nib << (8 * b + 4 * u);
+      }
+    }
     out[e] = v;
   }
 }
@@ -47,53 +68,51 @@ __global__ void pack_lut_kernel(const uint16_t* __restrict__ lut, Layout L,
     out[e] = e < (size_t)L.n * 16 ? lut[e] : (uint16_t)0;
 }
 
+// One thread per scale word: [panel][group][g][j], j = 2*half + (beta ? 1 : 0),
+// value = v(r) | v(r+16) << 16 with r = 32*panel + g + 8*half.
 __global__ void pack_scales_kernel(const uint16_t* __restrict__ alpha,
                                    const uint16_t* __restrict__ beta, Layout L,
                                    uint32_t* __restrict__ out) {
-  const size_t total = (size_t)L.n_pad * L.groups;
+  const size_t total = (size_t)L.panels * L.groups * 32;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
-    const int r16 = (int)(e % kTileRows);
-    const size_t tg = e / kTileRows;
-    const int grp = (int)(tg % L.groups);
-    const size_t tile = tg / L.groups;
-    const size_t row = tile * kTileRows + r16;
-    out[e] = row < (size_t)L.n ? ((uint32_t)alpha[row * L.groups + grp] |
-                                  ((uint32_t)beta[row * L.groups + grp] << 16))
-                               : 0u;
+    const int j = (int)(e & 3);
+    const int g = (int)((e >> 2) & 7);
+    const size_t pg = e >> 5;
+    const int grp = (int)(pg % L.groups);
+    const size_t panel = pg / L.groups;
+    const uint16_t* src = (j & 1) ? beta : alpha;
+    const size_t r0 = panel * kPanelRows + g + 8 * (j >> 1), r1 = r0 + 16;
+    uint32_t v = 0;
+    if (r0 < (size_t)L.n) v |= src[r0 * L.groups + grp];
+    if (r1 < (size_t)L.n) v |= (uint32_t)src[r1 * L.groups + grp] << 16;
+    out[e] = v;
   }
 }
 
-// One thread per packed 32-bit word: 8 weights (4 in row g, 4 in row g+8).
+// One thread per packed 32-bit word: 8 weights (two columns of four rows).
 __global__ void dequant_kernel(const uint8_t* __restrict__ packed, Layout L,
                                uint16_t* __restrict__ w) {
   const uint32_t* words = reinterpret_cast<const uint32_t*>(packed + L.w_off);
   const uint16_t* lutsec = reinterpret_cast<const uint16_t*>(packed + L.lut_off);
   const uint32_t* ab = reinterpret_cast<const uint32_t*>(packed + L.ab_off);
   const size_t total = (size_t)L.n_pad * L.k / 8;
-  const int col_off[4] = {0, 1, 2, 3};
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
-    const int step = (int)(e & 3);
-    const int lane = (int)((e >> 2) & 31);
-    const size_t tile_atom = e >> 7;
-    const int atom = (int)(tile_atom % L.katoms);
-    const size_t tile = tile_atom / L.katoms;
-    const int g = lane >> 2, t = lane & 3;
+    const WordPos q = word_pos(e, L.kchunks);
     const uint32_t word = words[e];
-    const int c = atom * kAtomK + t * 16 + step * 4;
-    for (int half = 0; half < 2; ++half) {
-      const int r16 = g + 8 * half;
-      const size_t row = tile * kTileRows + r16;
-      if (row >= (size_t)L.n) continue;
-      for (int i = 0; i < 4; ++i) {
-        const int col = c + col_off[i];
-        const uint32_t q = (word >> (16 * half + 4 * i)) & 0xF;
-        const uint32_t s = ab[(tile * L.groups + col / L.g) * kTileRows + r16];
-        const float a = bf16_bits_to_float(s & 0xFFFF);
-        const float b = bf16_bits_to_float(s >> 16);
-        const float v = fmaf(a, bf16_bits_to_float(lutsec[row * 16 + q]), b);   // one fp32 rounding
-        const __nv_bfloat16 h = __float2bfloat16_rn(v);                          // then bf16
+    for (int b = 0; b < 4; ++b) {
+      const int col = q.c0 + (b >> 1);
+      const int half = b & 1;
+      const uint32_t* s = ab + ((q.panel * L.groups + col / L.g) * 8 + q.g) * 4 + 2 * half;
+      for (int u = 0; u < 2; ++u) {
+        const size_t row = q.panel * kPanelRows + byte_row(q.g, b) + 16 * u;
+        if (row >= (size_t)L.n) continue;
+        const uint32_t idx = (word >> (8 * b + 4 * u)) & 0xFu;
+        const float a = bf16_bits_to_float((s[0] >> (16 * u)) & 0xFFFFu);
+        const float c = bf16_bits_to_float((s[1] >> (16 * u)) & 0xFFFFu);
+        const float v = fmaf(a, bf16_bits_to_float(lutsec[row * 16 + idx]), c);   // one fp32 rounding
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);                            // then bf16
         w[row * L.k + col] = *reinterpret_cast<const uint16_t*>(&h);
       }
     }
@@ -114,7 +133,7 @@ cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint1
       idx_nib, L, reinterpret_cast<uint32_t*>(packed + L.w_off));
   pack_lut_kernel<<<grid_for((size_t)L.n_pad * 16, th), th, 0, stream>>>(
       lut, L, reinterpret_cast<uint16_t*>(packed + L.lut_off));
-  pack_scales_kernel<<<grid_for((size_t)L.n_pad * L.groups, th), th, 0, stream>>>(
+  pack_scales_kernel<<<grid_for((size_t)L.panels * L.groups * 32, th), th, 0, stream>>>(
       alpha, beta, L, reinterpret_cast<uint32_t*>(packed + L.ab_off));
   return cudaGetLastError();
 }

@@ -30,11 +30,11 @@
 //  * Work split: a thread block (one per SM) owns a contiguous range of
 //    (32-row panel, 64-column chunk) units (stream-K). For each panel its
 //    consumer warps build the 16 row-pair tables (64 KB) once, then split the
-//    panel's chunks. A producer warp streams every consumer warp's weights and
-//    alpha/beta, two chunks per bulk copy, into per-warp rings of full/empty
-//    mbarriers; the consumers load their activation columns straight from L2
-//    (two 128-bit loads per chunk, one chunk ahead). No block-wide barrier
-//    inside a panel. The warps' fp32 tiles are summed in warp order; a panel
+//    panel's chunks. A producer warp streams every consumer warp's weights,
+//    four chunks (4 KB) per bulk copy, into per-warp rings of full/empty
+//    mbarriers; the consumers load their activation columns and alpha/beta
+//    straight from L2 (three 128-bit loads per chunk, one chunk ahead). No
+//    block-wide barrier inside a panel. The warps' fp32 tiles are summed in warp order; a panel
 //    split between thread blocks is finished by the last one to arrive, which
 //    sums the partials in thread-block order (deterministic; nothing waits on
 //    another thread block).
@@ -49,9 +49,12 @@ namespace any4 {
 namespace {
 
 constexpr int kMinUnitsPerCta = 32;
-constexpr int kPieceChunks = 2;                             // chunks per bulk copy
-constexpr int kSlotW = kPieceChunks * kChunkBytes;          // weights of one piece
-constexpr int kSlotBytes = kSlotW + kPieceChunks * kGroupScaleBytes;   // + up to 2 groups of alpha/beta
+// Weights stream in pieces of up to 4 chunks (4 KB), one bulk copy each: on
+// B200 a bulk copy costs ~100+ cycles of issue in the producer warp whatever
+// its size, so 1-2 KB copies cap the stream at 2-4 TB/s; 4 KB copies reach
+// 6-7 TB/s.
+constexpr int kPieceChunks = 4;
+constexpr int kSlotBytes = kPieceChunks * kChunkBytes;
 constexpr int kMiscBytes = 1024;                            // mbarriers and flags
 constexpr uint32_t kTabAddr = 131072;        // shared-window address of the row-pair tables
 constexpr uint32_t kTabBytes = 65536;        // 256 entries x 2 halves x 8 pairs x 4 copies x 4 B
@@ -65,7 +68,7 @@ template <int MODE>
 struct Cfg {
   static constexpr bool kTr = MODE == 2;
   static constexpr int kNt8 = MODE == 0 ? 1 : 2;                  // 8-column MMA tiles
-  static constexpr int kNW = MODE == 0 ? 16 : 8;                  // consumer warps
+  static constexpr int kNW = 8;                                   // consumer warps
   static constexpr int kThreads = (kNW + 2) * 32;                 // + producer and reducer warps
   static constexpr int kNF = kTr ? 16 : 4 * kNt8;                 // fp32 results per lane
   static constexpr int kNS = 3;                                   // ring depth (pieces)
@@ -246,22 +249,17 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     cur.start(P0, P1, u_lo, u_hi, kc, lane);
     if (lane >= NW) cur.panel = P1 + 1;   // lanes without a consumer warp
     const uint8_t* wbase = p.packed + p.w_off;
-    const uint8_t* abase = p.packed + p.ab_off;
     int issued = 0;   // pieces issued so far; piece q uses slot q % NS for the (q / NS)-th time
     while (cur.valid()) {
       const int slot = issued % NS;
       const int n = min(kPieceChunks, cur.cend - cur.c);
-      const int g_lo = (cur.c * kChunkCols) >> p.g_shift;
-      const int g_hi = ((cur.c + n) * kChunkCols - 1) >> p.g_shift;
       const uint32_t wbytes = (uint32_t)n * kChunkBytes;
-      const uint32_t sbytes = (uint32_t)(g_hi - g_lo + 1) * kGroupScaleBytes;
       if (issued >= NS)   // the consumer's release of the slot's previous use
         wait_bar(empty_bar(lane, slot), (uint32_t)(issued / NS - 1) & 1u, abort);
       if (*abort) break;
       const uint32_t fb = full_bar(lane, slot), dst = slot_addr(lane, slot);
-      mbar_arrive_expect_tx(fb, wbytes + sbytes);
+      mbar_arrive_expect_tx(fb, wbytes);
       bulk_g2s(dst, wbase + (((size_t)cur.panel * kc + cur.c) << 10), wbytes, fb);
-      bulk_g2s(dst + kSlotW, abase + (((size_t)cur.panel * p.groups + g_lo) << 7), sbytes, fb);
       ++issued;
       cur.c += n;
       cur.settle();
@@ -383,17 +381,75 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     selb1[h] = !ok ? 0x4444u : (g & 1) ? 0x3244u : 0x4432u;
     xmask[h] = ok ? 0xffffffffu : 0u;
   }
-  // words s = 0..7 of a chunk: columns 16t + 2s, +1 of the chunk
-  uint4 xn[NX][2];
-  auto load_x = [&](int c) {
+  // Per chunk, loaded from L2 one chunk ahead: the activation words (word
+  // s = 0..7 of tile h = component s & 3 of xn[h][s >> 2]; columns 16t + 2s, +1
+  // of the chunk) and this lane's alpha/beta pairs of the chunk's group.
+  const uint8_t* abase = p.packed + p.ab_off + 16 * g;
+  uint4 xn[NX][2], scn;
+  ChunkCursor<NW> xc;   // the chunk whose operands load next
+  xc.start(P0, P1, u_lo, u_hi, kc, warp);
+  auto next_operands = [&]() {
+    if (!xc.valid()) return;
+    const int c = xc.c;
 #pragma unroll
     for (int h = 0; h < NX; ++h) {
-      xn[h][0] = ld_nc_v4(xrow[h] + (size_t)c * kChunkCols);
-      xn[h][1] = ld_nc_v4(xrow[h] + (size_t)c * kChunkCols + 8);
+      const uint16_t* src = xrow[h] + (size_t)c * kChunkCols;
+      xn[h][0] = ld_nc_v4(src);
+      xn[h][1] = ld_nc_v4(src + 8);
+    }
+    scn = ld_nc_v4(abase + (((size_t)xc.panel * p.groups + ((c * kChunkCols) >> p.g_shift)) << 7));
+    ++xc.c;
+    xc.settle();
+  };
+
+  // decode + contract one chunk (8 steps) from its weight words, alpha/beta
+  // and activation words
+  float acc[NF / 4][4];   // one m16n8 fp32 tile per 4 results
+  auto chunk = [&](const uint4& wa, const uint4& wb, const uint4& sc, const uint32_t (&xw)[NX][8]) {
+    const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    if (!C::kTr) {
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        uint32_t a[4];
+        a[0] = lds32(prmt(w[s], baseA, 0x7604u));
+        a[1] = lds32(prmt(w[s], baseB, 0x7614u));
+        a[2] = lds32(prmt(w[s], baseA, 0x7624u));
+        a[3] = lds32(prmt(w[s], baseB, 0x7634u));
+        a[0] = fma_bf16x2(a[0], sc.x, sc.y);
+        a[2] = fma_bf16x2(a[2], sc.x, sc.y);
+        a[1] = fma_bf16x2(a[1], sc.z, sc.w);
+        a[3] = fma_bf16x2(a[3], sc.z, sc.w);
+#pragma unroll
+        for (int h = 0; h < NX; ++h)
+          mma_m16n8k16(acc[h], a, prmt(xw[h][s], 0u, selb0[h]), prmt(xw[h][s], 0u, selb1[h]));
+      }
+    } else {
+#pragma unroll
+      for (int s = 0; s < 8; s += 2) {
+        uint32_t e[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          e[u][0] = lds32(prmt(w[s + u], baseA, 0x7604u));
+          e[u][1] = lds32(prmt(w[s + u], baseB, 0x7614u));
+          e[u][2] = lds32(prmt(w[s + u], baseA, 0x7624u));
+          e[u][3] = lds32(prmt(w[s + u], baseB, 0x7634u));
+          e[u][0] = fma_bf16x2(e[u][0], sc.x, sc.y);
+          e[u][2] = fma_bf16x2(e[u][2], sc.x, sc.y);
+          e[u][1] = fma_bf16x2(e[u][1], sc.z, sc.w);
+          e[u][3] = fma_bf16x2(e[u][3], sc.z, sc.w);
+        }
+#pragma unroll
+        for (int tile = 0; tile < 2; ++tile) {
+          const uint32_t sel = tile ? 0x7632u : 0x5410u;
+          const uint32_t a[4] = {prmt(e[0][0], e[0][2], sel), prmt(e[0][1], e[0][3], sel),
+                                 prmt(e[1][0], e[1][2], sel), prmt(e[1][1], e[1][3], sel)};
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            mma_m16n8k16(acc[2 * tile + h], a, xw[h][s] & xmask[h], xw[h][s + 1] & xmask[h]);
+        }
+      }
     }
   };
-  ChunkCursor<NW> xc;   // the chunk whose activations load next
-  xc.start(P0, P1, u_lo, u_hi, kc, warp);
 
   int q = 0;   // pieces consumed; piece q sits in slot q % NS, phase (q / NS) & 1
 
@@ -418,104 +474,42 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     if (P == P0) {
       // activations, y and the workspace are touched only from here on
       asm volatile("griddepcontrol.wait;" ::: "memory");
-      if (xc.valid()) {
-        load_x(xc.c);
-        ++xc.c;
-        xc.settle();
-      }
+      next_operands();
     }
     consumer_sync(NCT);   // tables ready
 
-    float acc[NF];
 #pragma unroll
-    for (int i = 0; i < NF; ++i) acc[i] = 0.0f;
+    for (int i = 0; i < NF / 4; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
 
-    ChunkCursor<NW> mine;
-    mine.panel = P; mine.plast = P1; mine.u_lo = u_lo; mine.u_hi = u_hi; mine.kc = kc; mine.w = warp;
-    mine.open();
-    for (int pc = mine.c; pc < mine.cend; pc += kPieceChunks) {
-      const int n = min(kPieceChunks, mine.cend - pc);
-      const int g_lo = (pc * kChunkCols) >> p.g_shift;
+    int c0, c1;
+    {
+      ChunkCursor<NW> mine;
+      mine.panel = P; mine.u_lo = u_lo; mine.u_hi = u_hi; mine.kc = kc; mine.w = warp;
+      mine.open();
+      c0 = mine.c; c1 = mine.cend;
+    }
+    // pieces of up to kPieceChunks chunks from the warp's ring, chunk by chunk
+    for (int pc = c0; pc < c1; pc += kPieceChunks) {
+      const int n = min(kPieceChunks, c1 - pc);
       const int slot = q % NS;
-      const uint32_t sb = slot_addr(warp, slot);
+      const uint32_t sb = slot_addr(warp, slot) + 16u * lane;
       wait_bar(full_bar(warp, slot), (uint32_t)(q / NS) & 1u, abort);
+      ++q;
       for (int cc = 0; cc < n; ++cc) {
-        const int c = pc + cc;
-        uint4 xv[NX][2];
-#pragma unroll
-        for (int h = 0; h < NX; ++h) { xv[h][0] = xn[h][0]; xv[h][1] = xn[h][1]; }
-        if (xc.valid()) {   // next chunk's activations, one chunk ahead
-          load_x(xc.c);
-          ++xc.c;
-          xc.settle();
-        }
-        const uint32_t wsb = sb + (uint32_t)cc * kChunkBytes;
-        const uint4 wa = lds128(wsb + 16u * lane), wb = lds128(wsb + 512u + 16u * lane);
-        // alpha/beta pairs of (g, g+16) and (g+8, g+24) for this chunk's group
-        const uint4 sc = lds128(sb + kSlotW + ((uint32_t)(((c * kChunkCols) >> p.g_shift) - g_lo) << 7) +
-                                16u * g);
-        // release the slot once its last loads have landed (acc[0] depends on
-        // every load of the piece's earlier chunk)
-        if (cc == n - 1) mbar_arrive_after(empty_bar(warp, slot), wa.x, wb.x, sc.x, __float_as_uint(acc[0]));
-        const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        const uint4 wa = lds128(sb + (uint32_t)cc * kChunkBytes);
+        const uint4 wb = lds128(sb + (uint32_t)cc * kChunkBytes + 512u);
+        // release the slot once its last words are in registers
+        if (cc == n - 1) mbar_arrive_after(empty_bar(warp, slot), wa.x, wb.x, 0u, 0u);
         uint32_t xw[NX][8];
 #pragma unroll
         for (int h = 0; h < NX; ++h) {
-          xw[h][0] = xv[h][0].x; xw[h][1] = xv[h][0].y; xw[h][2] = xv[h][0].z; xw[h][3] = xv[h][0].w;
-          xw[h][4] = xv[h][1].x; xw[h][5] = xv[h][1].y; xw[h][6] = xv[h][1].z; xw[h][7] = xv[h][1].w;
+          xw[h][0] = xn[h][0].x; xw[h][1] = xn[h][0].y; xw[h][2] = xn[h][0].z; xw[h][3] = xn[h][0].w;
+          xw[h][4] = xn[h][1].x; xw[h][5] = xn[h][1].y; xw[h][6] = xn[h][1].z; xw[h][7] = xn[h][1].w;
         }
-        if (!C::kTr) {
-#pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            uint32_t a[4];
-            a[0] = lds32(prmt(w[s], baseA, 0x7604u));
-            a[1] = lds32(prmt(w[s], baseB, 0x7614u));
-            a[2] = lds32(prmt(w[s], baseA, 0x7624u));
-            a[3] = lds32(prmt(w[s], baseB, 0x7634u));
-            a[0] = fma_bf16x2(a[0], sc.x, sc.y);
-            a[2] = fma_bf16x2(a[2], sc.x, sc.y);
-            a[1] = fma_bf16x2(a[1], sc.z, sc.w);
-            a[3] = fma_bf16x2(a[3], sc.z, sc.w);
-#pragma unroll
-            for (int h = 0; h < NX; ++h) {
-              float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[4 * h]);
-              mma_m16n8k16(d, a, prmt(xw[h][s], 0u, selb0[h]), prmt(xw[h][s], 0u, selb1[h]));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < NX; ++h)
-#pragma unroll
-            for (int s = 0; s < 8; ++s) xw[h][s] &= xmask[h];
-#pragma unroll
-          for (int s = 0; s < 8; s += 2) {
-            uint32_t e[2][4];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              e[u][0] = lds32(prmt(w[s + u], baseA, 0x7604u));
-              e[u][1] = lds32(prmt(w[s + u], baseB, 0x7614u));
-              e[u][2] = lds32(prmt(w[s + u], baseA, 0x7624u));
-              e[u][3] = lds32(prmt(w[s + u], baseB, 0x7634u));
-              e[u][0] = fma_bf16x2(e[u][0], sc.x, sc.y);
-              e[u][2] = fma_bf16x2(e[u][2], sc.x, sc.y);
-              e[u][1] = fma_bf16x2(e[u][1], sc.z, sc.w);
-              e[u][3] = fma_bf16x2(e[u][3], sc.z, sc.w);
-            }
-#pragma unroll
-            for (int tile = 0; tile < 2; ++tile) {
-              const uint32_t sel = tile ? 0x7632u : 0x5410u;
-              const uint32_t a[4] = {prmt(e[0][0], e[0][2], sel), prmt(e[0][1], e[0][3], sel),
-                                     prmt(e[1][0], e[1][2], sel), prmt(e[1][1], e[1][3], sel)};
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                float(&d)[4] = *reinterpret_cast<float(*)[4]>(&acc[8 * tile + 4 * h]);
-                mma_m16n8k16(d, a, xw[h][s], xw[h][s + 1]);
-              }
-            }
-          }
-        }
+        const uint4 sc = scn;
+        next_operands();   // the next chunk's activations and alpha/beta
+        chunk(wa, wb, sc, xw);
       }
-      ++q;
     }
 
     // ---- hand the warp tiles to the reducer warp (double-buffered)
@@ -525,7 +519,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       float4* dst = reinterpret_cast<float4*>(tiles + (size_t)b * NW * 32 * NF + (size_t)(warp * 32 + lane) * NF);
 #pragma unroll
       for (int i = 0; i < NF / 4; ++i)
-        dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+        dst[i] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     }
     named_arrive(2 + b, NCT + 32);
     consumer_sync(NCT);   // every consumer is past its lookups: the tables are free

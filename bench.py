@@ -33,6 +33,10 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 GROUP = 128
+# DRAM bytes per algorithmic byte of the linear kernel, from one ncu capture
+# (profiles/linear_kernel_gate_14336x4096.md: 31,691,520 B read + 0 B written
+# for 31,690,752 algorithmic bytes). Set to None when the kernel changes.
+DRAM_PER_ALGO_BYTE = 31691520 / 31690752
 LAYERS = 32
 MS = (1, 16)
 FALLBACK_HBM_GBS = 6650.0
@@ -304,7 +308,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "us_per_call": ms_step * 1e3 / len(calls),
             "by_m": per_m,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak,
+                         "traffic": (DRAM_PER_ALGO_BYTE * step_bytes / len(calls)
+                                     if DRAM_PER_ALGO_BYTE is not None else None),
+                         "traffic_note": "dram bytes per launch: ncu dram__bytes_read+write of one "
+                                         "14336x4096 M=1 launch over its algorithmic bytes, times "
+                                         "this step's mean algorithmic bytes per launch",
                          "peak_source": f"{peak_kind} hbm_gbs", "kernel": "linear_kernel"},
             "gpu_launches": len(calls) * args.steps,
             "clocks": sampler.summary(),

@@ -60,6 +60,17 @@ import numpy as np
 from .bf16 import bf16_bits_to_f64, f32_to_bf16_bits, f64_to_bf16_bits, fma_to_f32
 
 INT4_GRID = np.arange(-8.0, 8.0)          # the fixed int4 integer map -8..7
+
+
+def int_grid(bits: int) -> np.ndarray:
+    """The signed integer map of a b-bit code: -2^(b-1) .. 2^(b-1)-1 (float64).
+
+    For b = 4 this is the int4 map -8..7 of the explainer's §一; the any3 and
+    any2 variants (named on the arXiv summary page) use the 3- and 2-bit maps
+    [reading].
+    """
+    h = 1 << (bits - 1)
+    return np.arange(-h, h, dtype=np.float64)
 _CHUNK_ELEMS = 1 << 19                     # rows per chunk = this // K
 
 
@@ -71,6 +82,7 @@ class Any4Tensors:
     alpha: np.ndarray
     beta: np.ndarray
     group: int
+    bits: int = 4          # indices use values < 2**bits; lut columns past that repeat
 
     @property
     def n(self) -> int:
@@ -102,11 +114,13 @@ def unpack_nibbles(idx_nib: np.ndarray) -> np.ndarray:
 
 # ----------------------------------------------------------- group scaling
 
-def group_scale(w_bits: np.ndarray, g: int):
+def group_scale(w_bits: np.ndarray, g: int, bits: int = 4):
     """Per-group alpha, beta (bf16 bits) and the scaled weights w_s (float64).
 
     Follows the group-scaling step (explainer §二.1): contiguous groups of g
-    columns in each row; asymmetric min-max onto [-8, 7].
+    columns in each row; asymmetric min-max onto [-8, 7] (for b bits onto
+    [-2^(b-1), 2^(b-1)-1], i.e. alpha = (max-min)/(2^b-1), beta = min +
+    2^(b-1) alpha [reading]).
     """
     w = bf16_bits_to_f64(w_bits)
     n, k = w.shape
@@ -115,9 +129,11 @@ def group_scale(w_bits: np.ndarray, g: int):
     wg = w.reshape(n, k // g, g)
     lo = wg.min(axis=2)
     hi = wg.max(axis=2)
-    alpha_bits = f64_to_bf16_bits((hi - lo) / 15.0)
+    levels = float((1 << bits) - 1)
+    half = float(1 << (bits - 1))
+    alpha_bits = f64_to_bf16_bits((hi - lo) / levels)
     alpha = bf16_bits_to_f64(alpha_bits)
-    beta_bits = f64_to_bf16_bits(lo + 8.0 * alpha)
+    beta_bits = f64_to_bf16_bits(lo + half * alpha)
     beta = bf16_bits_to_f64(beta_bits)
     a = alpha[:, :, None]
     safe = np.where(a == 0.0, 1.0, a)
@@ -141,12 +157,14 @@ def kmeans_weights(alpha_bits: np.ndarray, ex: np.ndarray, g: int) -> np.ndarray
 
 # ---------------------------------------------------------------- k-means
 
-def init_lut(ws: np.ndarray) -> np.ndarray:
-    """Initial 16-entry table per row (reading: distinct values or int4 grid)."""
-    lut = np.tile(INT4_GRID, (ws.shape[0], 1))
+def init_lut(ws: np.ndarray, bits: int = 4) -> np.ndarray:
+    """Initial 2^b-entry table per row (reading: distinct values or the
+    integer grid)."""
+    size = 1 << bits
+    lut = np.tile(int_grid(bits), (ws.shape[0], 1))
     for r in range(ws.shape[0]):
         u = np.unique(ws[r])
-        if u.size <= 16:
+        if u.size <= size:
             lut[r, :u.size] = u
             lut[r, u.size:] = u[-1]
     return lut
@@ -168,11 +186,11 @@ def m_step(ws: np.ndarray, c: np.ndarray, idx: np.ndarray, lut: np.ndarray) -> n
     values at exactly that value in float64. A cluster with sum(c) == 0 keeps
     its value.
     """
-    r = ws.shape[0]
-    slot = (np.arange(r)[:, None] * 16 + idx).ravel()
+    r, size = lut.shape
+    slot = (np.arange(r)[:, None] * size + idx).ravel()
     cur = np.take_along_axis(lut, idx.astype(np.int64), axis=1)
-    den = np.bincount(slot, weights=c.ravel(), minlength=r * 16).reshape(r, 16)
-    num = np.bincount(slot, weights=(c * (ws - cur)).ravel(), minlength=r * 16).reshape(r, 16)
+    den = np.bincount(slot, weights=c.ravel(), minlength=r * size).reshape(r, size)
+    num = np.bincount(slot, weights=(c * (ws - cur)).ravel(), minlength=r * size).reshape(r, size)
     out = lut.copy()
     nz = den > 0.0
     out[nz] = lut[nz] + num[nz] / den[nz]
@@ -185,14 +203,15 @@ def objective(ws: np.ndarray, c: np.ndarray, idx: np.ndarray, lut: np.ndarray) -
     return np.sum(c * (ws - v) ** 2, axis=1)
 
 
-def kmeans_rows(ws: np.ndarray, c: np.ndarray, iters: int = 10, history: bool = False):
-    """Weighted 1-D k-means with 16 centres for each row of ws.
+def kmeans_rows(ws: np.ndarray, c: np.ndarray, iters: int = 10, history: bool = False,
+                bits: int = 4):
+    """Weighted 1-D k-means with 2^bits (16 for any4) centres for each row of ws.
 
     Returns ``(idx, lut_bits)`` (and the per-row objective after every E and
     M step when ``history``): ``iters`` E/M rounds from ``init_lut``, then the
     table is rounded to bf16 and a last E-step runs against it.
     """
-    lut = init_lut(ws)
+    lut = init_lut(ws, bits)
     hist = []
     for _ in range(iters):
         idx = e_step(ws, lut)
@@ -209,11 +228,14 @@ def kmeans_rows(ws: np.ndarray, c: np.ndarray, iters: int = 10, history: bool = 
 
 
 def quantize(w_bits: np.ndarray, ex: np.ndarray, g: int = 128, iters: int = 10,
-             rows=None) -> Any4Tensors:
+             rows=None, bits: int = 4) -> Any4Tensors:
     """any4 quantization of a bf16 weight matrix (all rows, or ``rows`` only).
 
     Group scaling -> c = alpha * E|x| -> per-row weighted k-means, processed
-    in row chunks to bound memory.
+    in row chunks to bound memory. ``bits`` = 3 or 2 gives the any3 / any2
+    variants (8- and 4-entry tables); their tables are returned padded to 16
+    columns by repeating the last entry, so the same canonical tensors and
+    device layout serve every width.
     """
     w_bits = np.asarray(w_bits, dtype=np.uint16)
     if rows is not None:
@@ -226,14 +248,16 @@ def quantize(w_bits: np.ndarray, ex: np.ndarray, g: int = 128, iters: int = 10,
     step = max(1, _CHUNK_ELEMS // k)
     for r0 in range(0, n, step):
         r1 = min(n, r0 + step)
-        a_bits, b_bits, ws = group_scale(w_bits[r0:r1], g)
+        a_bits, b_bits, ws = group_scale(w_bits[r0:r1], g, bits)
         c = kmeans_weights(a_bits, ex, g)
-        idx, l_bits = kmeans_rows(ws, c, iters)
+        idx, l_bits = kmeans_rows(ws, c, iters, bits=bits)
         idx_nib[r0:r1] = pack_nibbles(idx)
-        lut[r0:r1] = l_bits
+        size = 1 << bits
+        lut[r0:r1, :size] = l_bits
+        lut[r0:r1, size:] = l_bits[:, size - 1:size]
         alpha[r0:r1] = a_bits
         beta[r0:r1] = b_bits
-    return Any4Tensors(idx_nib, lut, alpha, beta, g)
+    return Any4Tensors(idx_nib, lut, alpha, beta, g, bits)
 
 
 # ------------------------------------------------------------ dequantize

@@ -40,3 +40,35 @@ def nf4_levels() -> np.ndarray:
 
 def nf4_bf16_bits() -> np.ndarray:
     return f64_to_bf16_bits(nf4_levels())
+
+
+def fp4_e2m1_values() -> np.ndarray:
+    """The 16 values of the 4-bit floating-point element type E2M1 by code
+    0..15 (float64): bit 3 is the sign, bits 2..1 the exponent (bias 1),
+    bit 0 the mantissa; exponent 0 is subnormal (0 or 0.5).
+
+    The explainer's comparison table (§一) names FP4 among the 4-bit
+    baselines without defining it; E2M1 is read as the common FP4 element
+    format. Code 8 is -0.
+    """
+    out = np.empty(16, dtype=np.float64)
+    for q in range(16):
+        s, e, m = q >> 3, (q >> 1) & 3, q & 1
+        mag = m * 0.5 if e == 0 else 2.0 ** (e - 1) * (1.0 + 0.5 * m)
+        out[q] = -mag if s else mag
+    out[8] = -0.0
+    return out
+
+
+FORMATS = ("int4", "nf4", "fp4")
+
+
+def format_lut_bits(fmt: str) -> np.ndarray:
+    """bf16 bits of the fixed 16-entry table of a 4-bit baseline format."""
+    if fmt == "int4":
+        return f64_to_bf16_bits(int4_grid())
+    if fmt == "nf4":
+        return nf4_bf16_bits()
+    if fmt == "fp4":
+        return f64_to_bf16_bits(fp4_e2m1_values())
+    raise ValueError(fmt)

@@ -153,6 +153,37 @@ ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, in
 ANY4_API int any4_linear_noalloc(const uint16_t* x, const void* packed, int m, int n, int k,
                                  int group, uint16_t* y, any4_stream_t stream);
 
+/*
+ * Fixed-table 4-bit formats (explainer section 1, comparison table: int4,
+ * NF4 and FP4 against any4). Each is one 16-entry table shared by every row,
+ * so a weight in one of these formats is an any4 weight whose row tables are
+ * all equal, and it runs through any4_dequant and any4_linear unchanged.
+ *   ANY4_FORMAT_INT4  -8, -7, ..., 7 (code q -> q - 8)
+ *   ANY4_FORMAT_NF4   4-bit NormalFloat: 7 negative and 8 positive quantiles
+ *                     of the standard normal plus 0, in [-1, 1], ascending
+ *   ANY4_FORMAT_FP4   E2M1 element type: code bit 3 = sign, bits 2..1 =
+ *                     exponent (bias 1), bit 0 = mantissa; code 8 is -0
+ * Values are rounded to bf16 nearest-even.
+ */
+typedef enum { ANY4_FORMAT_INT4 = 1, ANY4_FORMAT_NF4 = 2, ANY4_FORMAT_FP4 = 3 } any4_format;
+
+/*
+ * any4_format_lut - the 16 bf16 values (bit patterns) of a format, by code.
+ * Host only, no GPU needed. lut: host array of 16 uint16_t written by the
+ * call. Returns ANY4_OK, or ANY4_EINVAL for a NULL lut or an unknown format.
+ */
+ANY4_API int any4_format_lut(int format, uint16_t* lut);
+
+/*
+ * any4_pack_format - any4_pack with the format's table in every row.
+ * idx_nib, alpha, beta, n, k, group, packed, packed_bytes and stream are as
+ * for any4_pack (the indices are the format's 4-bit codes); no LUT input.
+ * Returns as any4_pack; ANY4_EINVAL also for an unknown format.
+ */
+ANY4_API int any4_pack_format(int format, const uint8_t* idx_nib, const uint16_t* alpha,
+                              const uint16_t* beta, int n, int k, int group, void* packed,
+                              size_t packed_bytes, any4_stream_t stream);
+
 /* Static description of a status code (never NULL). */
 ANY4_API const char* any4_strerror(int status);
 

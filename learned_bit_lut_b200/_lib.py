@@ -37,13 +37,21 @@ lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_s
 lib.any4_linear.restype = _c_int
 lib.any4_linear_noalloc.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_linear_noalloc.restype = _c_int
+lib.any4_format_lut.argtypes = [_c_int, _p]
+lib.any4_format_lut.restype = _c_int
+lib.any4_pack_format.argtypes = [_c_int, _p, _p, _p, _c_int, _c_int, _c_int, _p, _c_size, _p]
+lib.any4_pack_format.restype = _c_int
 lib.any4_strerror.argtypes = [_c_int]
 lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
-            "any4_linear", "any4_linear_noalloc", "any4_strerror", "any4_last_cuda_error")
+            "any4_linear", "any4_linear_noalloc", "any4_format_lut", "any4_pack_format",
+            "any4_strerror", "any4_last_cuda_error")
+
+ANY4_FORMAT_INT4, ANY4_FORMAT_NF4, ANY4_FORMAT_FP4 = 1, 2, 3
+FORMATS = {"int4": ANY4_FORMAT_INT4, "nf4": ANY4_FORMAT_NF4, "fp4": ANY4_FORMAT_FP4}
 
 ANY4_OK, ANY4_EINVAL, ANY4_EALIGN, ANY4_ESHAPE, ANY4_EWORKSPACE, ANY4_ECUDA = 0, -1, -2, -3, -4, -5
 
@@ -160,6 +168,37 @@ def any4_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, g
     _check(lib.any4_linear_noalloc(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k,
                                    group, _dev(out, "out", 2, (m, n)), _stream(x.device)))
     return out
+
+
+def _format_code(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def any4_format_lut(fmt) -> list:
+    """The 16 bf16 bit patterns of a fixed-table format ("int4", "nf4", "fp4"),
+    by code. Host only."""
+    buf = (ctypes.c_uint16 * 16)()
+    _check(lib.any4_format_lut(_format_code(fmt), ctypes.cast(buf, _p)))
+    return [int(v) for v in buf]
+
+
+def any4_pack_format(fmt, idx_nib: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+                     group: int, packed: torch.Tensor | None = None) -> torch.Tensor:
+    """Fixed-table format codes + alpha/beta -> device-layout buffer; the
+    format's table goes to every row, so any4_dequant / any4_linear apply."""
+    n, k2 = idx_nib.shape
+    k = 2 * k2
+    size = any4_packed_bytes(n, k, group)
+    if size == 0:
+        raise Any4Error(ANY4_ESHAPE)
+    dev = idx_nib.device
+    if packed is None:
+        packed = torch.empty(size, dtype=torch.uint8, device=dev)
+    _check(lib.any4_pack_format(_format_code(fmt), _dev(idx_nib, "idx_nib", 1, (n, k2)),
+                                _dev(alpha, "alpha", 2, (n, k // group)),
+                                _dev(beta, "beta", 2, (n, k // group)), n, k, group,
+                                _dev(packed, "packed", 1), packed.numel(), _stream(dev)))
+    return packed
 
 
 def any4_strerror(status: int) -> str:

@@ -45,6 +45,10 @@ int current_sm_count(int* sms) {
 
 }  // namespace
 
+namespace any4 {
+int record_cuda_error(cudaError_t e) { return fail_cuda(e); }
+}  // namespace any4
+
 extern "C" {
 
 size_t any4_packed_bytes(int n, int k, int group) {

@@ -14,6 +14,17 @@ cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint1
                         const uint16_t* beta, const Layout& L, uint8_t* packed,
                         cudaStream_t stream);
 
+// Pack with the same table in every row (fixed-table formats).
+cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
+                              const uint16_t* alpha, const uint16_t* beta, const Layout& L,
+                              uint8_t* packed, cudaStream_t stream);
+
+// Keeps e for any4_last_cuda_error() on this host thread; returns ANY4_ECUDA.
+int record_cuda_error(cudaError_t e);
+
+// The 16 bf16 values of a fixed-table format (any4_format); false if unknown.
+bool format_table(int format, uint16_t (&lut)[16]);
+
 cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream);
 

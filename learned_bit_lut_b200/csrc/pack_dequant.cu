@@ -68,14 +68,31 @@ __global__ void pack_lut_kernel(const uint16_t* __restrict__ lut, Layout L,
     out[e] = e < (size_t)L.n * 16 ? lut[e] : (uint16_t)0;
 }
 
+// The same 16-entry table in every row (fixed-table formats).
+struct Table16 {
+  uint16_t v[16];
+};
+
+__global__ void pack_lut_fixed_kernel(Table16 t, Layout L, uint16_t* __restrict__ out) {
+  const size_t total = (size_t)L.n_pad * 16;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x)
+    out[e] = e < (size_t)L.n * 16 ? t.v[e & 15] : (uint16_t)0;
+}
+
 // One thread per scale word: [panel][group][g][j], j = 2*half + (beta ? 1 : 0),
 // value = v(r) | v(r+16) << 16 with r = 32*panel + g + 8*half.
 __global__ void pack_scales_kernel(const uint16_t* __restrict__ alpha,
                                    const uint16_t* __restrict__ beta, Layout L,
                                    uint32_t* __restrict__ out) {
   const size_t total = (size_t)L.panels * L.groups * 32;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+  const size_t padded = (L.total - L.ab_off) / 4;   // the section's tail padding is written as 0
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < padded;
        e += (size_t)gridDim.x * blockDim.x) {
+    if (e >= total) {
+      out[e] = 0u;
+      continue;
+    }
     const int j = (int)(e & 3);
     const int g = (int)((e >> 2) & 7);
     const size_t pg = e >> 5;
@@ -133,7 +150,22 @@ cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint1
       idx_nib, L, reinterpret_cast<uint32_t*>(packed + L.w_off));
   pack_lut_kernel<<<grid_for((size_t)L.n_pad * 16, th), th, 0, stream>>>(
       lut, L, reinterpret_cast<uint16_t*>(packed + L.lut_off));
-  pack_scales_kernel<<<grid_for((size_t)L.panels * L.groups * 32, th), th, 0, stream>>>(
+  pack_scales_kernel<<<grid_for((L.total - L.ab_off) / 4, th), th, 0, stream>>>(
+      alpha, beta, L, reinterpret_cast<uint32_t*>(packed + L.ab_off));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
+                              const uint16_t* alpha, const uint16_t* beta, const Layout& L,
+                              uint8_t* packed, cudaStream_t stream) {
+  const int th = 256;
+  Table16 t;
+  for (int q = 0; q < 16; ++q) t.v[q] = lut[q];
+  pack_weights_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(
+      idx_nib, L, reinterpret_cast<uint32_t*>(packed + L.w_off));
+  pack_lut_fixed_kernel<<<grid_for((size_t)L.n_pad * 16, th), th, 0, stream>>>(
+      t, L, reinterpret_cast<uint16_t*>(packed + L.lut_off));
+  pack_scales_kernel<<<grid_for((L.total - L.ab_off) / 4, th), th, 0, stream>>>(
       alpha, beta, L, reinterpret_cast<uint32_t*>(packed + L.ab_off));
   return cudaGetLastError();
 }

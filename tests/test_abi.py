@@ -6,7 +6,10 @@ import re
 
 import pytest
 
+import numpy as np
+
 import learned_bit_lut_b200 as a4
+import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -71,3 +74,27 @@ def test_strerror_covers_all_codes():
     for code in (0, -1, -2, -3, -4, -5):
         assert a4.any4_strerror(code).startswith("ANY4_")
     assert "unknown" in a4.any4_strerror(7)
+
+
+def test_format_tables_match_oracle():
+    # host-side tables of the fixed formats, built independently of the oracle
+    for fmt in oracle.FORMATS:
+        lib_bits = np.array(a4.any4_format_lut(fmt), dtype=np.uint16)
+        np.testing.assert_array_equal(lib_bits, oracle.format_lut_bits(fmt))
+
+
+def test_format_lut_rejects_unknown_format():
+    buf = (ctypes.c_uint16 * 16)()
+    assert a4.lib.any4_format_lut(0, ctypes.cast(buf, ctypes.c_void_p)) == a4.ANY4_EINVAL
+    assert a4.lib.any4_format_lut(a4.ANY4_FORMAT_NF4, None) == a4.ANY4_EINVAL
+
+
+def test_pack_format_rejects_bad_arguments():
+    dummy = ctypes.c_void_p(256)
+    # unknown format, null pointer, bad shape, misaligned buffer: all before any launch
+    assert a4.lib.any4_pack_format(9, dummy, dummy, dummy, 32, 64, 64, dummy, 1 << 20, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_pack_format(1, None, dummy, dummy, 32, 64, 64, dummy, 1 << 20, None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_pack_format(1, dummy, dummy, dummy, 33, 64, 64, dummy, 1 << 20, None) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_pack_format(1, dummy, dummy, dummy, 32, 64, 64, ctypes.c_void_p(258), 1 << 20,
+                                   None) == a4.ANY4_EALIGN
+    assert a4.lib.any4_pack_format(1, dummy, dummy, dummy, 32, 64, 64, dummy, 16, None) == a4.ANY4_EWORKSPACE

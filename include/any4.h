@@ -154,6 +154,35 @@ ANY4_API int any4_linear_noalloc(const uint16_t* x, const void* packed, int m, i
                                  int group, uint16_t* y, any4_stream_t stream);
 
 /*
+ * any4_quantize - the any4 quantizer on the GPU (explainer sections 2.1 and
+ * 2.2): group scaling, then per-row weighted k-means with 2^bits centres.
+ *
+ *   w        [N][K] bf16 weights (device).
+ *   ex       [K] float64 E|x| per input channel from a calibration sample
+ *            (section 2.1); the k-means weight of column k is alpha * ex[k].
+ *   bits     4 (any4), 3 (any3) or 2 (any2); iters: E/M rounds, 0..1000
+ *            (10 in this library's tests).
+ *   outputs  the canonical tensors any4_pack consumes: idx_nib [N][K/2]
+ *            (even column in the low nibble; codes < 2^bits), lut [N][16]
+ *            bf16 (2^bits learned entries, padded by repeating the last),
+ *            alpha and beta [N][K/G] bf16.
+ * Group scaling is asymmetric min-max onto [-2^(bits-1), 2^(bits-1)-1]:
+ * alpha = (max-min)/(2^bits-1), beta = min + 2^(bits-1)*alpha, both rounded
+ * to bf16. The start table is the row's distinct scaled values when there
+ * are at most 2^bits of them, else the integer map; E-step ties go to the
+ * lowest index; an empty cluster keeps its value; after the rounds the table
+ * is rounded to bf16 and a last E-step assigns against it. All arithmetic is
+ * float64 with each cluster sum taken in column order, so the output is a
+ * deterministic function of the inputs. One thread per row: meant for
+ * model preparation, not for the per-token path.
+ * Returns ANY4_OK, ANY4_EINVAL (null pointer, bits or iters out of range) or
+ * ANY4_ESHAPE (N, K, G as for any4_pack).
+ */
+ANY4_API int any4_quantize(const uint16_t* w, const double* ex, int n, int k, int group, int bits,
+                           int iters, uint8_t* idx_nib, uint16_t* lut, uint16_t* alpha,
+                           uint16_t* beta, any4_stream_t stream);
+
+/*
  * Fixed-table 4-bit formats (explainer section 1, comparison table: int4,
  * NF4 and FP4 against any4). Each is one 16-entry table shared by every row,
  * so a weight in one of these formats is an any4 weight whose row tables are

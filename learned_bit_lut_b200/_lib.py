@@ -41,13 +41,16 @@ lib.any4_format_lut.argtypes = [_c_int, _p]
 lib.any4_format_lut.restype = _c_int
 lib.any4_pack_format.argtypes = [_c_int, _p, _p, _p, _c_int, _c_int, _c_int, _p, _c_size, _p]
 lib.any4_pack_format.restype = _c_int
+lib.any4_quantize.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p]
+lib.any4_quantize.restype = _c_int
 lib.any4_strerror.argtypes = [_c_int]
 lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
-            "any4_linear", "any4_linear_noalloc", "any4_format_lut", "any4_pack_format",
+            "any4_linear", "any4_linear_noalloc", "any4_quantize", "any4_format_lut",
+            "any4_pack_format",
             "any4_strerror", "any4_last_cuda_error")
 
 ANY4_FORMAT_INT4, ANY4_FORMAT_NF4, ANY4_FORMAT_FP4 = 1, 2, 3
@@ -168,6 +171,24 @@ def any4_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, g
     _check(lib.any4_linear_noalloc(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k,
                                    group, _dev(out, "out", 2, (m, n)), _stream(x.device)))
     return out
+
+
+def any4_quantize(w: torch.Tensor, ex: torch.Tensor, group: int, bits: int = 4,
+                  iters: int = 10):
+    """GPU any4 quantizer: bf16 W (N x K) and float64 E|x| (K) -> the canonical
+    tensors (idx_nib, lut, alpha, beta) as int16/uint8 device tensors."""
+    n, k = w.shape
+    dev = w.device
+    idx_nib = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+    lut = torch.empty((n, 16), dtype=torch.int16, device=dev)
+    alpha = torch.empty((n, k // group), dtype=torch.int16, device=dev)
+    beta = torch.empty((n, k // group), dtype=torch.int16, device=dev)
+    if ex.dtype != torch.float64:
+        raise ValueError("ex must be float64")
+    _check(lib.any4_quantize(_dev(w, "w", 2, (n, k)), _dev(ex, "ex", 8, (k,)), n, k, group, bits,
+                             iters, _dev(idx_nib, "idx_nib", 1), _dev(lut, "lut", 2),
+                             _dev(alpha, "alpha", 2), _dev(beta, "beta", 2), _stream(dev)))
+    return idx_nib, lut, alpha, beta
 
 
 def _format_code(fmt) -> int:

@@ -19,6 +19,11 @@ cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
                               const uint16_t* alpha, const uint16_t* beta, const Layout& L,
                               uint8_t* packed, cudaStream_t stream);
 
+// any4 quantizer (group scaling + weighted k-means), one thread per row.
+cudaError_t launch_quantize(const uint16_t* w, const double* ex, int n, int k, int g, int bits,
+                            int iters, uint8_t* idx_nib, uint16_t* lut, uint16_t* alpha,
+                            uint16_t* beta, cudaStream_t stream);
+
 // Keeps e for any4_last_cuda_error() on this host thread; returns ANY4_ECUDA.
 int record_cuda_error(cudaError_t e);
 

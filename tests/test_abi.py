@@ -98,3 +98,14 @@ def test_pack_format_rejects_bad_arguments():
     assert a4.lib.any4_pack_format(1, dummy, dummy, dummy, 32, 64, 64, ctypes.c_void_p(258), 1 << 20,
                                    None) == a4.ANY4_EALIGN
     assert a4.lib.any4_pack_format(1, dummy, dummy, dummy, 32, 64, 64, dummy, 16, None) == a4.ANY4_EWORKSPACE
+
+
+def test_quantize_rejects_bad_arguments():
+    d = ctypes.c_void_p(256)
+    q = a4.lib.any4_quantize
+    assert q(None, d, 32, 64, 64, 4, 10, d, d, d, d, None) == a4.ANY4_EINVAL
+    assert q(d, d, 32, 64, 64, 5, 10, d, d, d, d, None) == a4.ANY4_EINVAL      # bits
+    assert q(d, d, 32, 64, 64, 1, 10, d, d, d, d, None) == a4.ANY4_EINVAL
+    assert q(d, d, 32, 64, 64, 4, -1, d, d, d, d, None) == a4.ANY4_EINVAL      # iters
+    assert q(d, d, 31, 64, 64, 4, 10, d, d, d, d, None) == a4.ANY4_ESHAPE
+    assert q(d, d, 32, 64, 96, 4, 10, d, d, d, d, None) == a4.ANY4_ESHAPE

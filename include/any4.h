@@ -123,9 +123,14 @@ ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
  * Each weight is dequantized as w_hat = fma(alpha, LUT[idx], beta) in bf16
  * (fma.rn.bf16x2: the exact value rounded once to bf16) and contracted on the
  * tensor cores (mma.sync m16n8k16) with fp32 accumulation; the fp32 result
- * is rounded to bf16 nearest-even. Blocks split along K are reduced in a
- * fixed order, so the result is deterministic. No thread block ever waits on
- * another one.
+ * is rounded to bf16 nearest-even. Output rows split along K between thread
+ * blocks (at most one block per SM, all resident at once) are finished by the
+ * block that holds their first columns: it waits for the others' fp32
+ * partials and adds them in a fixed order, so the result is deterministic.
+ * Every wait in the kernel is bounded (~2 s); if one gives up, the kernel
+ * completes without hanging and the first 32-bit word of the workspace's
+ * reserved area (byte offset 65536*4) is set non-zero. It is zero after
+ * every normal call.
  */
 ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);

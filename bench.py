@@ -33,9 +33,10 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 GROUP = 128
-# DRAM bytes per algorithmic byte of the linear kernel, from one ncu capture
-# (profiles/linear_kernel_gate_14336x4096.md: 31,691,520 B read + 0 B written
-# for 31,690,752 algorithmic bytes). Set to None when the kernel changes.
+# DRAM bytes per algorithmic byte of the linear kernel, from one ncu capture of
+# a 14336x4096, M=1, G=128 launch (dram__bytes_read.sum 31,691,520 B,
+# dram__bytes_write.sum 0 B, for 31,690,752 algorithmic bytes). Set to None
+# when the kernel changes.
 DRAM_PER_ALGO_BYTE = 31691520 / 31690752
 LAYERS = 32
 MS = (1, 16)

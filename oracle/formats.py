@@ -26,12 +26,9 @@ from .bf16 import bf16_bits_to_f64, f64_to_bf16_bits
 from .tables import format_lut_bits, fp4_e2m1_values, nf4_bf16_bits
 
 
-def quantize_format(w_bits: np.ndarray, fmt: str, g: int = 128) -> Any4Tensors:
-    """Quantize a bf16 weight matrix to a fixed-table format (canonical tensors)."""
-    w_bits = np.asarray(w_bits, dtype=np.uint16)
+def _quantize_format_rows(w_bits: np.ndarray, fmt: str, g: int):
     n, k = w_bits.shape
-    table_bits = format_lut_bits(fmt)
-    table = bf16_bits_to_f64(table_bits)
+    table = bf16_bits_to_f64(format_lut_bits(fmt))
     if fmt == "int4":
         alpha_bits, beta_bits, ws = group_scale(w_bits, g)
     else:
@@ -44,7 +41,22 @@ def quantize_format(w_bits: np.ndarray, fmt: str, g: int = 128) -> Any4Tensors:
         safe = np.where(a == 0.0, 1.0, a)
         ws = np.where(a == 0.0, 0.0, w / safe).reshape(n, k)
     idx = e_step(ws, np.tile(table, (n, 1)))
-    return Any4Tensors(pack_nibbles(idx), np.tile(table_bits, (n, 1)), alpha_bits, beta_bits, g)
+    return pack_nibbles(idx), alpha_bits, beta_bits
+
+
+def quantize_format(w_bits: np.ndarray, fmt: str, g: int = 128) -> Any4Tensors:
+    """Quantize a bf16 weight matrix to a fixed-table format (canonical
+    tensors), in row chunks to bound memory."""
+    w_bits = np.asarray(w_bits, dtype=np.uint16)
+    n, k = w_bits.shape
+    idx_nib = np.empty((n, k // 2), dtype=np.uint8)
+    alpha = np.empty((n, k // g), dtype=np.uint16)
+    beta = np.empty((n, k // g), dtype=np.uint16)
+    step = max(1, (1 << 19) // k)
+    for r0 in range(0, n, step):
+        r1 = min(n, r0 + step)
+        idx_nib[r0:r1], alpha[r0:r1], beta[r0:r1] = _quantize_format_rows(w_bits[r0:r1], fmt, g)
+    return Any4Tensors(idx_nib, np.tile(format_lut_bits(fmt), (n, 1)), alpha, beta, g)
 
 
 __all__ = ["quantize_format", "format_lut_bits", "fp4_e2m1_values", "nf4_bf16_bits"]

@@ -37,7 +37,7 @@ GROUP = 128
 # a 14336x4096, M=1, G=128 launch (dram__bytes_read.sum 31,691,520 B,
 # dram__bytes_write.sum 0 B, for 31,690,752 algorithmic bytes). Set to None
 # when the kernel changes.
-DRAM_PER_ALGO_BYTE = 31691520 / 31690752
+DRAM_PER_ALGO_BYTE = None
 LAYERS = 32
 MS = (1, 16)
 FALLBACK_HBM_GBS = 6650.0

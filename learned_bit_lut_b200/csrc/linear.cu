@@ -56,9 +56,10 @@ constexpr int kMinUnitsPerCta = 32;
 constexpr int kPieceChunks = 4;
 constexpr int kSlotBytes = kPieceChunks * kChunkBytes;
 constexpr int kMiscBytes = 1024;                            // mbarriers and flags
-constexpr uint32_t kTabAddr = 131072;        // shared-window address of the row-pair tables
+constexpr uint32_t kTabAddr = 65536;         // shared-window address of the row-pair tables
 constexpr uint32_t kTabBytes = 65536;        // 256 entries x 2 halves x 8 pairs x 4 copies x 4 B
-constexpr uint32_t kRedAddr = kTabAddr + kTabBytes;
+constexpr uint32_t kHighAddr = kTabAddr + kTabBytes;   // ring overflow and warp tiles
+constexpr uint32_t kMaxWindowBase = 8192;    // the dynamic window starts below this
 constexpr long long kWaitLimitCycles = 4000000000ll;   // ~2 s: then the kernel records a timeout
 constexpr int kConsumerBar = 1;              // named barrier of the consumer warps
 
@@ -68,15 +69,19 @@ template <int MODE>
 struct Cfg {
   static constexpr bool kTr = MODE == 2;
   static constexpr int kNt8 = MODE == 0 ? 1 : 2;                  // 8-column MMA tiles
-  static constexpr int kNW = 8;                                   // consumer warps
+  static constexpr int kNW = MODE == 0 ? 16 : MODE == 1 ? 12 : 8; // consumer warps
   static constexpr int kThreads = (kNW + 2) * 32;                 // + producer and reducer warps
   static constexpr int kNF = kTr ? 16 : 4 * kNt8;                 // fp32 results per lane
-  static constexpr int kNS = 3;                                   // ring depth (pieces)
-  static constexpr int kRingBytes = kNW * kNS * kSlotBytes;
+  static constexpr int kNS = MODE == 2 ? 3 : 2;                   // ring depth (pieces)
+  static constexpr int kSlots = kNW * kNS;
   static constexpr int kTileBytes = kNW * 32 * kNF * 4;           // the warps' fp32 tiles of a panel
-  static constexpr int kSmemBytes = (int)kRedAddr + 2 * kTileBytes;   // covers any window base
+  // ring slots go below the tables while they fit (for the highest window
+  // base), the rest above them, followed by the two buffers of warp tiles
+  static constexpr int kLowSlotsMin = ((int)kTabAddr - (int)kMaxWindowBase - kMiscBytes) / kSlotBytes;
+  static constexpr int kHighSlotsMax = kSlots > kLowSlotsMin ? kSlots - kLowSlotsMin : 0;
+  static constexpr int kSmemBytes = (int)kHighAddr + kHighSlotsMax * kSlotBytes + 2 * kTileBytes;
   // everything below the tables, for a window that starts within 8 KB
-  static_assert(8192 + kMiscBytes + kRingBytes <= (int)kTabAddr, "rings overlap the tables");
+  static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 struct Params {
@@ -203,12 +208,14 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   const uint32_t base = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // Shared window: [mbarriers, flags][per-warp rings] ... [row-pair tables at
-  // kTabAddr][two buffers of warp tiles]. The dynamic window starts at a small
-  // fixed offset, so the rings fit below the tables; if they ever do not,
+  // Shared window: [mbarriers, flags][ring slots][row-pair tables at 64 KB]
+  // [remaining ring slots][two buffers of warp tiles]. The dynamic window
+  // starts at a small fixed offset; if it ever starts higher than planned,
   // record it and leave before touching anything else.
   const uint32_t ring0 = base + kMiscBytes;
-  if (ring0 + (uint32_t)C::kRingBytes > kTabAddr) {
+  const int n_low = min(C::kSlots, (int)((kTabAddr - ring0) / kSlotBytes));
+  const uint32_t tiles_addr = kHighAddr + (uint32_t)(C::kSlots - n_low) * kSlotBytes;
+  if (base > kMaxWindowBase || tiles_addr + 2u * C::kTileBytes > base + (uint32_t)C::kSmemBytes) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) atomicOr(p.status, 2u);
     return;
@@ -216,8 +223,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + 1016);
   auto full_bar = [&](int w, int s) { return base + (uint32_t)(w * NS + s) * 16u; };
   auto empty_bar = [&](int w, int s) { return base + (uint32_t)(w * NS + s) * 16u + 8u; };
-  auto slot_addr = [&](int w, int s) { return ring0 + (uint32_t)(w * NS + s) * kSlotBytes; };
-  float* tiles = reinterpret_cast<float*>(smem + (kRedAddr - base));   // [2][NW][32][NF]
+  auto slot_addr = [&](int w, int s) {
+    const int i = w * NS + s;
+    return i < n_low ? ring0 + (uint32_t)i * kSlotBytes : kHighAddr + (uint32_t)(i - n_low) * kSlotBytes;
+  };
+  float* tiles = reinterpret_cast<float*>(smem + (tiles_addr - base));   // [2][NW][32][NF]
 
   const long long U = p.units;
   const int kc = p.kc;
@@ -342,7 +352,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 
   // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
   // 8*blh .. 8*blh+7; every entry goes to its four bank copies
-  constexpr int kBuildPer = 512 / NCT;
+  constexpr int kBuildPer = (512 + NCT - 1) / NCT;   // 512 tasks per panel
   const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off);
   // this thread's LUT values of the panel being built (lw/lh) and of the
   // next one (nw/nh), loaded a full panel ahead
@@ -352,6 +362,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 #pragma unroll
     for (int r = 0; r < kBuildPer; ++r) {
       const int task = tid + r * NCT;
+      if (task >= 512) break;
       const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
       const int br0 = (brp & 7) + 8 * (brp >> 3);
       dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
@@ -458,6 +469,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 #pragma unroll
     for (int r = 0; r < kBuildPer; ++r) {
       const int task = tid + r * NCT;
+      if (task >= 512) break;
       const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
       const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
       const uint32_t L[4] = {lw[r].x, lw[r].y, lw[r].z, lw[r].w};

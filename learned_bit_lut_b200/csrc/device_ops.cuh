@@ -39,6 +39,31 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
+// 128-bit load of read-only data kept in L1 ahead of other lines (evict_last).
+__device__ __forceinline__ uint4 ld_keep_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// 128-bit load of read-only data used once (not allocated in L1).
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// 16-bit load of read-only data used once (not allocated in L1), zero-extended.
+__device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
+  unsigned short v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
 // 16-bit load of read-only data, zero-extended.
 __device__ __forceinline__ uint32_t ld_nc_u16(const void* p) {
   unsigned short v;

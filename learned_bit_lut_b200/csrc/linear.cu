@@ -349,6 +349,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 
   // =========================== consumer warps ==============================
   const int g = lane >> 2, t = lane & 3;
+  // Row-pair modes keep the activations in L1 (evict_last) and stream the LUT
+  // and alpha/beta past it, loading alpha/beta once per group: on B200 this
+  // keeps the L1 misses, which cost several data-pipe wavefronts each, off the
+  // activation loads.
+  constexpr bool kRowPair = !C::kTr;
 
   // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
   // 8*blh .. 8*blh+7; every entry goes to its four bank copies
@@ -365,8 +370,13 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       if (task >= 512) break;
       const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
       const int br0 = (brp & 7) + 8 * (brp >> 3);
-      dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
-      dh[r] = ld_nc_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+      if (kRowPair) {
+        dw[r] = ld_stream_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
+        dh[r] = ld_stream_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+      } else {
+        dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
+        dh[r] = ld_nc_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+      }
     }
   };
   load_lut(P0, lw, lh);
@@ -397,6 +407,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   // of the chunk) and this lane's alpha/beta pairs of the chunk's group.
   const uint8_t* abase = p.packed + p.ab_off + 16 * g;
   uint4 xn[NX][2], scn;
+  int last_grp = -1;
   ChunkCursor<NW> xc;   // the chunk whose operands load next
   xc.start(P0, P1, u_lo, u_hi, kc, warp);
   auto next_operands = [&]() {
@@ -405,10 +416,16 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 #pragma unroll
     for (int h = 0; h < NX; ++h) {
       const uint16_t* src = xrow[h] + (size_t)c * kChunkCols;
-      xn[h][0] = ld_nc_v4(src);
-      xn[h][1] = ld_nc_v4(src + 8);
+      xn[h][0] = kRowPair ? ld_keep_v4(src) : ld_nc_v4(src);
+      xn[h][1] = kRowPair ? ld_keep_v4(src + 8) : ld_nc_v4(src + 8);
     }
-    scn = ld_nc_v4(abase + (((size_t)xc.panel * p.groups + ((c * kChunkCols) >> p.g_shift)) << 7));
+    const int grp = xc.panel * p.groups + ((c * kChunkCols) >> p.g_shift);
+    if (!kRowPair) {
+      scn = ld_nc_v4(abase + ((size_t)grp << 7));
+    } else if (grp != last_grp) {   // a new group: its alpha/beta (read once, not kept in L1)
+      scn = ld_stream_v4(abase + ((size_t)grp << 7));
+      last_grp = grp;
+    }
     ++xc.c;
     xc.settle();
   };

@@ -102,13 +102,20 @@ ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t*
  * (the launch is sized by the device's SM count); 0 if the shape is not
  * accepted. The workspace holds a fixed header of 65536 arrival counters (one
  * per possible 16-row tile) and a reserved 256-byte area, then the fp32
- * partial sums of output blocks split along K between thread blocks.
+ * partial sums of output blocks split along K between thread blocks. For
+ * M > 16 (prefill) the header is followed by a bf16 N x K scratch for the
+ * dequantized weight instead (N*K*2 bytes, rounded up to 256).
  */
 ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 
 /*
  * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
  *
+ *   m          tokens, 1 .. 2^20. M <= 16 (decode, explainer section 3's
+ *              batch 1-16) runs the fused dequant-and-contract kernel below;
+ *              M > 16 (prefill) dequantizes W once into the workspace (the
+ *              bit-exact any4_dequant values) and runs a tensor-core GEMM
+ *              (tcgen05, fp32 accumulation in tensor memory).
  *   x          [M][K] bf16 activations, row-major, 16-byte aligned.
  *   packed     the any4_pack output for W (N x K, group G).
  *   y          [M][N] bf16 output, row-major, 4-byte aligned.

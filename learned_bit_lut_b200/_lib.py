@@ -146,7 +146,8 @@ def workspace_for(m: int, n: int, k: int, group: int, device: torch.device) -> t
 def any4_linear(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: int,
                 out: torch.Tensor | None = None,
                 workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """y = x . W_hat^T for bf16 x (M x K, M <= 16) -> y (M x N, bf16)."""
+    """y = x . W_hat^T for bf16 x (M x K) -> y (M x N, bf16). M <= 16 runs the
+    fused decode kernel, M > 16 the dequantize-then-GEMM prefill path."""
     m = x.shape[0]
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)

@@ -80,7 +80,7 @@ int any4_dequant(const void* packed, int n, int k, int group, uint16_t* w, any4_
 }
 
 size_t any4_linear_workspace_bytes(int m, int n, int k, int group) {
-  if (m < 1 || m > 16 || !any4::shape_ok(n, k, group)) return 0;
+  if (m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group)) return 0;
   int sms = 0;
   if (current_sm_count(&sms) != ANY4_OK) return 0;
   return any4::plan_linear(m, any4::make_layout(n, k, group), sms).workspace_bytes;
@@ -89,7 +89,7 @@ size_t any4_linear_workspace_bytes(int m, int n, int k, int group) {
 int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream) {
   if (!x || !packed || !y || !workspace) return ANY4_EINVAL;
-  if (m < 1 || m > 16 || !any4::shape_ok(n, k, group)) return ANY4_ESHAPE;
+  if (m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group)) return ANY4_ESHAPE;
   if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(y, 4) || !aligned(workspace, 16))
     return ANY4_EALIGN;
   int sms = 0;

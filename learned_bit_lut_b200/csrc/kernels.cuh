@@ -44,9 +44,16 @@ constexpr size_t kCountersBytes = (size_t)kMaxTiles * sizeof(unsigned);
 constexpr size_t kHeaderBytes = kCountersBytes + 256;
 constexpr unsigned kStatusWaitTimeout = 1u;
 
+// M > 16 (prefill): bf16 W_hat scratch at prefill_scratch_offset() of the
+// workspace, then a tcgen05 GEMM (prefill.cu).
+size_t prefill_scratch_offset();
+size_t prefill_workspace_bytes(const Layout& L);
+cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
+                           void* workspace, int num_sms, cudaStream_t stream);
+
 // Launch geometry of any4_linear for one shape on one device.
 struct LinearPlan {
-  int mode;             // 0: M <= 4, 1: M <= 8 (row-pair operands); 2: M <= 16 (row operands)
+  int mode;             // 0: M <= 4, 1: M <= 8 (row-pair operands); 2: M <= 16 (row operands); 3: M > 16
   int nf;               // fp32 results per lane and panel
   long long units;      // panels x K/64 chunks
   int ctas;             // persistent thread blocks (one per SM at most)

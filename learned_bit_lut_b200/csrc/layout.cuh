@@ -46,6 +46,7 @@ constexpr int kChunkBytes = 1024;
 constexpr int kGroupScaleBytes = 128;   // one panel, one group
 constexpr int kAlign = 256;
 constexpr int kMaxRows = 1 << 20;
+constexpr int kMaxTokens = 1 << 20;     // M of any4_linear (M > 16 takes the prefill GEMM)
 
 struct Layout {
   int n, k, g;

@@ -597,6 +597,12 @@ cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t st
 
 LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   LinearPlan pl{};
+  if (m > 16) {   // prefill: dequantized W scratch + tensor-core GEMM
+    pl.mode = 3;
+    pl.workspace_bytes = prefill_workspace_bytes(L);
+    pl.ctas = num_sms;
+    return pl;
+  }
   pl.mode = m <= 4 ? 0 : m <= 8 ? 1 : 2;
   pl.nf = pl.mode == 0 ? 4 : pl.mode == 1 ? 8 : 16;
   pl.units = (long long)L.panels * L.kchunks;
@@ -612,6 +618,7 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
 cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout& L, int m,
                           uint16_t* y, void* workspace, const LinearPlan& plan,
                           cudaStream_t stream) {
+  if (plan.mode == 3) return launch_prefill(x, packed, L, m, y, workspace, plan.ctas, stream);
   cudaError_t e = allow_large_smem();
   if (e != cudaSuccess) return e;
   Params p{};

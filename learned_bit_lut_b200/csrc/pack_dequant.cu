@@ -136,6 +136,59 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, Layout L,
   }
 }
 
+// Tiled dequant: one thread block per (panel, 8 chunks = 512 columns). The
+// block decodes its words into a shared [32 rows][512 columns] bf16 tile
+// (same fp32 fma + round-to-nearest-even as dequant_kernel) and writes each
+// row segment with 16-byte stores, so the N x K output is written coalesced.
+constexpr int kDqChunks = 8;
+constexpr int kDqRow = kDqChunks * kChunkCols + 8;   // bf16 per tile row (16-byte pad)
+
+__global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __restrict__ packed, Layout L,
+                                                           uint16_t* __restrict__ w) {
+  __shared__ __align__(16) uint16_t tile[kPanelRows * kDqRow];
+  __shared__ uint16_t lut[kPanelRows * 16];
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(packed + L.w_off);
+  const uint16_t* lutsec = reinterpret_cast<const uint16_t*>(packed + L.lut_off);
+  const uint32_t* ab = reinterpret_cast<const uint32_t*>(packed + L.ab_off);
+  const int P = blockIdx.y;
+  const int c_begin = blockIdx.x * kDqChunks;
+  const int nch = min(kDqChunks, L.kchunks - c_begin);
+  for (int i = threadIdx.x; i < kPanelRows * 16; i += blockDim.x)
+    lut[i] = lutsec[(size_t)P * kPanelRows * 16 + i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < nch * 256; e += blockDim.x) {
+    const int cl = e >> 8, wi = e & 255;
+    const int i = wi & 3, ln = (wi >> 2) & 31, h = wi >> 7;
+    const int g = ln >> 2, t = ln & 3;
+    const int c0 = 16 * t + 2 * (4 * h + i);   // column within the chunk
+    const int col0 = (c_begin + cl) * kChunkCols + c0;
+    const uint32_t word = words[((size_t)P * L.kchunks + c_begin + cl) * 256 + wi];
+    const uint32_t* sc = ab + (((size_t)P * L.groups + col0 / L.g) * 8 + g) * 4;
+    for (int b = 0; b < 4; ++b) {
+      const int half = b & 1;
+      const uint32_t sa = sc[2 * half], sb = sc[2 * half + 1];
+      for (int u = 0; u < 2; ++u) {
+        const int r = byte_row(g, b) + 16 * u;
+        const uint32_t idx = (word >> (8 * b + 4 * u)) & 0xFu;
+        const float a = bf16_bits_to_float((sa >> (16 * u)) & 0xFFFFu);
+        const float c = bf16_bits_to_float((sb >> (16 * u)) & 0xFFFFu);
+        const float v = fmaf(a, bf16_bits_to_float(lut[r * 16 + idx]), c);   // one fp32 rounding
+        const __nv_bfloat16 hv = __float2bfloat16_rn(v);                       // then bf16
+        tile[r * kDqRow + cl * kChunkCols + c0 + (b >> 1)] = *reinterpret_cast<const uint16_t*>(&hv);
+      }
+    }
+  }
+  __syncthreads();
+  const int units = nch * kChunkCols / 8;   // 16-byte units per row
+  for (int i = threadIdx.x; i < kPanelRows * units; i += blockDim.x) {
+    const int r = i / units, u = i % units;
+    const size_t row = (size_t)P * kPanelRows + r;
+    if (row >= (size_t)L.n) continue;
+    const uint4 v = *reinterpret_cast<const uint4*>(&tile[r * kDqRow + u * 8]);
+    *reinterpret_cast<uint4*>(w + row * L.k + (size_t)c_begin * kChunkCols + u * 8) = v;
+  }
+}
+
 static int grid_for(size_t work, int threads) {
   size_t b = (work + threads - 1) / threads;
   if (b > 65535u * 8u) b = 65535u * 8u;
@@ -173,7 +226,12 @@ cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
 cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream) {
   const int th = 256;
-  dequant_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(packed, L, w);
+  if ((reinterpret_cast<uintptr_t>(w) & 15) == 0) {   // 16-byte stores need a 16-byte aligned w
+    const dim3 grid((L.kchunks + kDqChunks - 1) / kDqChunks, L.panels);
+    dequant_tile_kernel<<<grid, th, 0, stream>>>(packed, L, w);
+  } else {
+    dequant_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(packed, L, w);
+  }
   return cudaGetLastError();
 }
 

@@ -1,0 +1,341 @@
+// any4_linear for M > 16 (prefill): y = x . W_hat^T as a tensor-core GEMM.
+//
+// Beyond the explainer's batch 1-16 regime (10100.com article 149119421,
+// section 3: tinygemm runs small batches on the tensor cores) the product is
+// compute bound, so the path is:
+//   1. dequantize W into a bf16 N x K scratch (in the caller's workspace) with
+//      the bit-exact w_hat = fma(alpha, LUT[idx], beta) of sections 2-2.1
+//      (dequant_tile_kernel in pack_dequant.cu), then
+//   2. run a tcgen05 GEMM on it: D (128 weight rows x 256 tokens, fp32 in
+//      tensor memory) += W_hat tile (128 x 64, shared memory) . x tile^T
+//      (256 x 64, shared memory), both operands brought in by TMA with the
+//      128-byte swizzle, 4 pipeline stages, two accumulators so the epilogue
+//      of one tile overlaps the main loop of the next.
+// Dequantizing on the fly into shared memory instead would cost about two
+// instructions per weight on B200 (lookup, scale, store), while tensor memory
+// holds at most 512 tokens of fp32 accumulators per 128 rows: the decode
+// would then bound the GEMM at roughly a third of the tensor-core rate. The
+// separate pass costs about 2.5 bytes of memory traffic per weight once per
+// call instead.
+//
+// Warps: 0 = TMA producer, 1 = MMA issuer (and tensor-memory owner),
+// 2-5 = epilogue (warp w reads tensor-memory lanes 32*(w%4) .. +31).
+// Every mbarrier wait is bounded (~2 s); a timeout sets the workspace status
+// word and the block winds down.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <atomic>
+
+#include "kernels.cuh"
+
+namespace any4 {
+
+namespace {
+
+constexpr int kBM = 128;                       // weight rows per tile (MMA M)
+constexpr int kBN = 256;                       // tokens per tile (MMA N)
+constexpr int kBK = 64;                        // K per stage: one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kAStageBytes = kBM * kBK * 2;    // 16 KB
+constexpr int kBStageBytes = kBN * kBK * 2;    // 32 KB
+constexpr int kStageBytes = kAStageBytes + kBStageBytes;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kAccCols = kBN;             // fp32 columns per accumulator
+constexpr uint32_t kTmemCols = 2 * kAccCols;   // two accumulators
+constexpr int kGemmSmem = kStages * kStageBytes + 1024 + 1024;   // stages, control, alignment
+constexpr long long kGemmWaitCycles = 4000000000ll;
+
+// tcgen05 instruction descriptor, kind::f16: D fp32, A and B bf16, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+struct GemmCtl {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_arrive_one(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait; false when the block is aborting or the wait timed out.
+__device__ __forceinline__ bool gemm_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kGemmWaitCycles) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusWaitTimeout);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// arrives once on `bar` when every tcgen05.mma this thread issued so far is complete
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %3, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(accumulate), "r"(kIdesc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_x32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
+                        uint16_t* __restrict__ y, int m, int n, int k, unsigned* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;   // swizzle atoms need 1024-byte alignment
+  GemmCtl* ctl = reinterpret_cast<GemmCtl*>(smem_raw + (sbase - raw) + kStages * kStageBytes);
+  auto sa = [&](int s) { return sbase + (uint32_t)s * kStageBytes; };
+  auto sb = [&](int s) { return sbase + (uint32_t)s * kStageBytes + kAStageBytes; };
+  volatile int* abort_flag = &ctl->abort_flag;
+
+  const int n_tiles = (n + kBM - 1) / kBM, m_tiles = (m + kBN - 1) / kBN;
+  const int tiles = n_tiles * m_tiles, kch = k / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_addr(&ctl->full[s]), 1);    // TMA expect_tx arrival + bytes
+      mbar_init(smem_addr(&ctl->empty[s]), 1);   // tcgen05.commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_addr(&ctl->acc_full[b]), 1);    // tcgen05.commit
+      mbar_init(smem_addr(&ctl->acc_empty[b]), 4);   // one arrival per epilogue warp
+    }
+    ctl->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&ctl->tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl->tmem_base;
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // x (and the dequantized W) are ready
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
+        const int nt = tile / m_tiles, mt = tile % m_tiles;
+        for (int kc = 0; kc < kch; ++kc, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (it >= kStages &&
+              !gemm_wait(smem_addr(&ctl->empty[s]), ph ^ 1u, abort_flag, status))
+            break;
+          const uint32_t fb = smem_addr(&ctl->full[s]);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          tma_load_2d(sa(s), &wmap, kc * kBK, nt * kBM, fb);
+          tma_load_2d(sb(s), &xmap, kc * kBK, mt * kBN, fb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int it = 0, tcount = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
+        const int b = tcount & 1;
+        const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
+        if (tcount >= 2 && !gemm_wait(smem_addr(&ctl->acc_empty[b]), aph ^ 1u, abort_flag, status))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)b * kAccCols;
+        for (int kc = 0; kc < kch; ++kc, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+          if (!gemm_wait(smem_addr(&ctl->full[s]), ph, abort_flag, status)) break;
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(sa(s)), bd = sw128_desc(sb(s));
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)   // 16 columns = 32 bytes = 2 descriptor units
+            tc_mma(d, ad + 2u * (uint64_t)kk, bd + 2u * (uint64_t)kk, (kc | kk) != 0 ? 1u : 0u);
+          tc_commit(smem_addr(&ctl->empty[s]));   // the stage is free once these MMAs are done
+        }
+        tc_commit(smem_addr(&ctl->acc_full[b]));
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;   // tensor-memory lane quarter of this warp
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
+      const int nt = tile / m_tiles, mt = tile % m_tiles;
+      const int b = tcount & 1;
+      const uint32_t ph = (uint32_t)(tcount >> 1) & 1u;
+      if (!gemm_wait(smem_addr(&ctl->acc_full[b]), ph, abort_flag, status)) break;
+      tc_fence_after();
+      const int row = nt * kBM + 32 * q + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)b * kAccCols;
+#pragma unroll 1
+      for (int j = 0; j < kBN / 32; ++j) {
+        uint32_t v[32];
+        tc_ld_x32(tbase + 32u * (uint32_t)j, v);
+        tc_wait_ld();
+        const int m0 = mt * kBN + 32 * j;
+        if (row < n) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (m0 + i < m) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+              y[(size_t)(m0 + i) * n + row] = *reinterpret_cast<const uint16_t*>(&h);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_one(smem_addr(&ctl->acc_empty[b]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<void*> fn{nullptr};
+  void* f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn.store(f, std::memory_order_release);
+  }
+  return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// rows x cols bf16 matrix (row-major), boxes of box_rows x 64 columns, 128-byte swizzle
+bool encode_bf16_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t allow_gemm_smem() {
+  static std::atomic<unsigned long long> done_mask{0};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done_mask.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(prefill_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_relaxed);
+  return e;
+}
+
+}  // namespace
+
+size_t prefill_scratch_offset() { return kHeaderBytes; }
+
+size_t prefill_workspace_bytes(const Layout& L) {
+  return kHeaderBytes + align_up((size_t)L.n * L.k * 2, kAlign);
+}
+
+cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
+                           void* workspace, int num_sms, cudaStream_t stream) {
+  cudaError_t e = allow_gemm_smem();
+  if (e != cudaSuccess) return e;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  uint16_t* what = reinterpret_cast<uint16_t*>(ws + prefill_scratch_offset());
+  e = launch_dequant(packed, L, what, stream);   // bf16 W_hat, N x K
+  if (e != cudaSuccess) return e;
+  CUtensorMap wmap, xmap;
+  if (!encode_bf16_map(&wmap, what, L.n, L.k, kBM) || !encode_bf16_map(&xmap, x, m, L.k, kBN))
+    return cudaErrorInvalidValue;
+  const int tiles = ((L.n + kBM - 1) / kBM) * ((m + kBN - 1) / kBN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  unsigned* status = reinterpret_cast<unsigned*>(ws + kCountersBytes);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, wmap, xmap, y, m, L.n, L.k, status);
+}
+
+}  // namespace any4

@@ -1,0 +1,88 @@
+"""GPU parity of the prefill path (M > 16): the bf16 W_hat scratch must equal
+any4_dequant bit for bit, and y must meet the linear layer's acceptance bar
+and the tight elementwise bar (the GEMM contracts the same bf16 weights with
+fp32 accumulation). Shapes cover one tile, ragged token and row tails, K not
+a multiple of the 64-column stage count of a tile, every group size, and the
+Llama-3-8B MLP shapes at full size (sampled rows)."""
+import numpy as np
+import pytest
+import torch
+
+import learned_bit_lut_b200 as a4
+import synth
+from gpu_util import bf16_dev, bits_host, check_linear, mixed, pack_dev, quantized, require_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+STATUS_OFFSET = 65536 * 4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+    torch.cuda.set_device(0)
+
+
+@pytest.mark.parametrize("n,k,g,m", [(256, 512, 128, 17), (256, 512, 128, 64), (16, 64, 64, 17),
+                                     (1024, 4096, 128, 256), (160, 2112, 64, 300),
+                                     (4096, 1024, 256, 33), (48, 1024, 1024, 513), (272, 1536, 512, 257)])
+def test_prefill_shapes(n, k, g, m):
+    q, s = quantized(n, k, g, layer=f"pre{n}x{k}", iters=4)
+    x = synth.activations_bf16(m, s, 7, layer=f"pre{n}x{k}")
+    ws = a4.workspace_for(m, n, k, g, torch.device("cuda:0"))
+    y = a4.any4_linear(bf16_dev(x), pack_dev(q), n, k, g, workspace=ws)
+    torch.cuda.synchronize()
+    check_linear(y, x, q)
+    assert int(ws[STATUS_OFFSET:STATUS_OFFSET + 4].view(torch.int32)[0]) == 0
+
+
+@pytest.mark.parametrize("shape,m", [((14336, 4096), 512), ((4096, 14336), 384)])
+def test_prefill_llama3_8b_mlp_sampled(shape, m):
+    n, k = shape
+    rows = sample_rows(n, 48, seed=n + 1)
+    q, s = mixed(n, k, 128, rows, layer=f"pmlp{n}x{k}")
+    x = synth.activations_bf16(m, s, 8, layer=f"pmlp{n}x{k}")
+    y = a4.any4_linear(bf16_dev(x), pack_dev(q), n, k, 128)
+    check_linear(y, x, q, rows)
+
+
+def test_prefill_scratch_is_the_dequantized_weight():
+    n, k, g, m = 1024, 2048, 128, 40
+    q, s = quantized(n, k, g, layer="pscratch", iters=4)
+    x = synth.activations_bf16(m, s, 9, layer="pscratch")
+    packed = pack_dev(q)
+    ws = a4.workspace_for(m, n, k, g, torch.device("cuda:0"))
+    a4.any4_linear(bf16_dev(x), packed, n, k, g, workspace=ws)
+    w = a4.any4_dequant(packed, n, k, g)
+    torch.cuda.synchronize()
+    off = STATUS_OFFSET + 256
+    scratch = ws[off:off + n * k * 2].view(torch.int16).view(n, k)
+    assert torch.equal(scratch, w.view(torch.int16))
+
+
+def test_prefill_repeatable_and_guard_rows_untouched():
+    n, k, g, m = 512, 1024, 128, 100
+    q, s = quantized(n, k, g, layer="pguard", iters=4)
+    x = bf16_dev(synth.activations_bf16(m, s, 10, layer="pguard"))
+    packed = pack_dev(q)
+    buf = torch.full((m + 2, n), 7, dtype=torch.int16, device="cuda:0")
+    out = buf.view(torch.bfloat16)[1:m + 1]
+    a4.any4_linear(x, packed, n, k, g, out=out)
+    first = bits_host(out).copy()
+    a4.any4_linear(x, packed, n, k, g, out=out)
+    torch.cuda.synchronize()
+    assert np.array_equal(first, bits_host(out))
+    assert torch.all(buf[0] == 7) and torch.all(buf[m + 1] == 7)
+
+
+def test_prefill_workspace_size():
+    n, k, g = 4096, 4096, 128
+    need = a4.any4_linear_workspace_bytes(17, n, k, g)
+    assert need >= STATUS_OFFSET + 256 + n * k * 2
+    x = torch.zeros((17, k), dtype=torch.bfloat16, device="cuda:0")
+    y = torch.empty((17, n), dtype=torch.bfloat16, device="cuda:0")
+    packed = torch.zeros(a4.any4_packed_bytes(n, k, g), dtype=torch.uint8, device="cuda:0")
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device="cuda:0")
+    rc = a4.lib.any4_linear(x.data_ptr(), packed.data_ptr(), 17, n, k, g, y.data_ptr(), ws.data_ptr(),
+                            ws.numel(), None)
+    assert rc == a4.ANY4_EWORKSPACE

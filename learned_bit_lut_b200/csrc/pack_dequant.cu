@@ -146,42 +146,57 @@ constexpr int kDqRow = kDqChunks * kChunkCols + 8;   // bf16 per tile row (16-by
 __global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __restrict__ packed, Layout L,
                                                            uint16_t* __restrict__ w) {
   __shared__ __align__(16) uint16_t tile[kPanelRows * kDqRow];
-  __shared__ uint16_t lut[kPanelRows * 16];
+  __shared__ float lut[kPanelRows * 16];
   const uint32_t* words = reinterpret_cast<const uint32_t*>(packed + L.w_off);
   const uint16_t* lutsec = reinterpret_cast<const uint16_t*>(packed + L.lut_off);
   const uint32_t* ab = reinterpret_cast<const uint32_t*>(packed + L.ab_off);
   const int P = blockIdx.y;
   const int c_begin = blockIdx.x * kDqChunks;
   const int nch = min(kDqChunks, L.kchunks - c_begin);
-  for (int i = threadIdx.x; i < kPanelRows * 16; i += blockDim.x)
-    lut[i] = lutsec[(size_t)P * kPanelRows * 16 + i];
+  // word j of this thread: e = threadIdx.x + 256 j (chunk j of the strip, word
+  // threadIdx.x of the chunk); its weights and scales are loaded before the
+  // table barrier so the loads overlap
+  const int wi = threadIdx.x;
+  const int i = wi & 3, ln = (wi >> 2) & 31, h = wi >> 7;
+  const int g = ln >> 2, t = ln & 3;
+  const int c0 = 16 * t + 2 * (4 * h + i);   // column within a chunk
+  uint32_t word[kDqChunks];
+  uint4 sc[kDqChunks];
+#pragma unroll
+  for (int j = 0; j < kDqChunks; ++j) {
+    if (j < nch) {
+      const int col0 = (c_begin + j) * kChunkCols + c0;
+      word[j] = __ldg(words + ((size_t)P * L.kchunks + c_begin + j) * 256 + wi);
+      sc[j] = __ldg(reinterpret_cast<const uint4*>(ab + (((size_t)P * L.groups + col0 / L.g) * 8 + g) * 4));
+    }
+  }
+  for (int e = threadIdx.x; e < kPanelRows * 16; e += blockDim.x)
+    lut[e] = bf16_bits_to_float(lutsec[(size_t)P * kPanelRows * 16 + e]);
   __syncthreads();
-  for (int e = threadIdx.x; e < nch * 256; e += blockDim.x) {
-    const int cl = e >> 8, wi = e & 255;
-    const int i = wi & 3, ln = (wi >> 2) & 31, h = wi >> 7;
-    const int g = ln >> 2, t = ln & 3;
-    const int c0 = 16 * t + 2 * (4 * h + i);   // column within the chunk
-    const int col0 = (c_begin + cl) * kChunkCols + c0;
-    const uint32_t word = words[((size_t)P * L.kchunks + c_begin + cl) * 256 + wi];
-    const uint32_t* sc = ab + (((size_t)P * L.groups + col0 / L.g) * 8 + g) * 4;
-    for (int b = 0; b < 4; ++b) {
-      const int half = b & 1;
-      const uint32_t sa = sc[2 * half], sb = sc[2 * half + 1];
-      for (int u = 0; u < 2; ++u) {
-        const int r = byte_row(g, b) + 16 * u;
-        const uint32_t idx = (word >> (8 * b + 4 * u)) & 0xFu;
-        const float a = bf16_bits_to_float((sa >> (16 * u)) & 0xFFFFu);
-        const float c = bf16_bits_to_float((sb >> (16 * u)) & 0xFFFFu);
-        const float v = fmaf(a, bf16_bits_to_float(lut[r * 16 + idx]), c);   // one fp32 rounding
-        const __nv_bfloat16 hv = __float2bfloat16_rn(v);                       // then bf16
-        tile[r * kDqRow + cl * kChunkCols + c0 + (b >> 1)] = *reinterpret_cast<const uint16_t*>(&hv);
+#pragma unroll
+  for (int j = 0; j < kDqChunks; ++j) {
+    if (j < nch) {
+      const uint32_t sw[4] = {sc[j].x, sc[j].y, sc[j].z, sc[j].w};
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = g + 8 * half + 16 * u;
+          const float a = bf16_bits_to_float((sw[2 * half] >> (16 * u)) & 0xFFFFu);
+          const float c = bf16_bits_to_float((sw[2 * half + 1] >> (16 * u)) & 0xFFFFu);
+          const uint32_t i0 = (word[j] >> (8 * half + 4 * u)) & 0xFu;         // column c0
+          const uint32_t i1 = (word[j] >> (8 * (half + 2) + 4 * u)) & 0xFu;   // column c0 + 1
+          // one fp32 rounding each, then bf16 nearest-even
+          const __nv_bfloat162 v = __floats2bfloat162_rn(fmaf(a, lut[r * 16 + i0], c), fmaf(a, lut[r * 16 + i1], c));
+          *reinterpret_cast<__nv_bfloat162*>(&tile[r * kDqRow + j * kChunkCols + c0]) = v;
+        }
       }
     }
   }
   __syncthreads();
   const int units = nch * kChunkCols / 8;   // 16-byte units per row
-  for (int i = threadIdx.x; i < kPanelRows * units; i += blockDim.x) {
-    const int r = i / units, u = i % units;
+  for (int e = threadIdx.x; e < kPanelRows * units; e += blockDim.x) {
+    const int r = e / units, u = e % units;
     const size_t row = (size_t)P * kPanelRows + r;
     if (row >= (size_t)L.n) continue;
     const uint4 v = *reinterpret_cast<const uint4*>(&tile[r * kDqRow + u * 8]);

@@ -143,6 +143,28 @@ ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, in
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream);
 
 /*
+ * any3 / any2: the same calls for b = 3 or 2 bits per index (the lower-bit
+ * variants named in the abstract of the "any4: Learned 4-bit Numeric
+ * Representation for LLMs" summary page). The canonical inputs are as for
+ * any4_pack, with every index < 2^b (an 8- or 4-entry table per row; only the
+ * first 2^b LUT entries are read, the rest may be anything); any4_quantize
+ * with bits = 3 or 2 produces them. The packed buffer stores each row pair's
+ * two indices as one 2b-bit code, densely (N*K*b/8 bytes of indices) and is
+ * only valid for the *_bits calls with the same b. bits = 4 is the same as
+ * the plain calls. Workspace sizes are those of any4_linear_workspace_bytes.
+ * Errors as for the plain calls, plus ANY4_ESHAPE for bits not in {2, 3, 4}.
+ */
+ANY4_API size_t any4_packed_bytes_bits(int bits, int n, int k, int group);
+ANY4_API int any4_pack_bits(int bits, const uint8_t* idx_nib, const uint16_t* lut,
+                            const uint16_t* alpha, const uint16_t* beta, int n, int k, int group,
+                            void* packed, size_t packed_bytes, any4_stream_t stream);
+ANY4_API int any4_dequant_bits(int bits, const void* packed, int n, int k, int group, uint16_t* w,
+                               any4_stream_t stream);
+ANY4_API int any4_linear_bits(int bits, const uint16_t* x, const void* packed, int m, int n, int k,
+                              int group, uint16_t* y, void* workspace, size_t workspace_bytes,
+                              any4_stream_t stream);
+
+/*
  * any4_linear_noalloc - any4_linear for callers that cannot allocate device
  * memory. The source pages have no counterpart of this call; it exists for
  * callers such as operators running inside a serving runtime that owns all

@@ -43,6 +43,14 @@ lib.any4_pack_format.argtypes = [_c_int, _p, _p, _p, _c_int, _c_int, _c_int, _p,
 lib.any4_pack_format.restype = _c_int
 lib.any4_quantize.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _c_int, _p, _p, _p, _p, _p]
 lib.any4_quantize.restype = _c_int
+lib.any4_packed_bytes_bits.argtypes = [_c_int, _c_int, _c_int, _c_int]
+lib.any4_packed_bytes_bits.restype = _c_size
+lib.any4_pack_bits.argtypes = [_c_int, _p, _p, _p, _p, _c_int, _c_int, _c_int, _p, _c_size, _p]
+lib.any4_pack_bits.restype = _c_int
+lib.any4_dequant_bits.argtypes = [_c_int, _p, _c_int, _c_int, _c_int, _p, _p]
+lib.any4_dequant_bits.restype = _c_int
+lib.any4_linear_bits.argtypes = [_c_int, _p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
+lib.any4_linear_bits.restype = _c_int
 lib.any4_strerror.argtypes = [_c_int]
 lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
@@ -50,8 +58,8 @@ lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
             "any4_linear", "any4_linear_noalloc", "any4_quantize", "any4_format_lut",
-            "any4_pack_format",
-            "any4_strerror", "any4_last_cuda_error")
+            "any4_pack_format", "any4_packed_bytes_bits", "any4_pack_bits", "any4_dequant_bits",
+            "any4_linear_bits", "any4_strerror", "any4_last_cuda_error")
 
 ANY4_FORMAT_INT4, ANY4_FORMAT_NF4, ANY4_FORMAT_FP4 = 1, 2, 3
 FORMATS = {"int4": ANY4_FORMAT_INT4, "nf4": ANY4_FORMAT_NF4, "fp4": ANY4_FORMAT_FP4}
@@ -113,6 +121,51 @@ def any4_pack(idx_nib: torch.Tensor, lut: torch.Tensor, alpha: torch.Tensor, bet
                          _dev(beta, "beta", 2, (n, k // group)), n, k, group,
                          _dev(packed, "packed", 1), packed.numel(), _stream(dev)))
     return packed
+
+
+def any4_packed_bytes_bits(bits: int, n: int, k: int, group: int) -> int:
+    return lib.any4_packed_bytes_bits(bits, n, k, group)
+
+
+def any4_pack_bits(bits: int, idx_nib: torch.Tensor, lut: torch.Tensor, alpha: torch.Tensor,
+                   beta: torch.Tensor, group: int, packed: torch.Tensor | None = None) -> torch.Tensor:
+    """any3 / any2 (bits = 3 / 2; 4 = any4): canonical tensors with indices
+    < 2^bits (as nibbles) -> densely packed device-layout buffer."""
+    n, k2 = idx_nib.shape
+    k = 2 * k2
+    size = any4_packed_bytes_bits(bits, n, k, group)
+    if size == 0:
+        raise Any4Error(ANY4_ESHAPE)
+    dev = idx_nib.device
+    if packed is None:
+        packed = torch.empty(size, dtype=torch.uint8, device=dev)
+    _check(lib.any4_pack_bits(bits, _dev(idx_nib, "idx_nib", 1, (n, k2)), _dev(lut, "lut", 2, (n, 16)),
+                              _dev(alpha, "alpha", 2, (n, k // group)),
+                              _dev(beta, "beta", 2, (n, k // group)), n, k, group,
+                              _dev(packed, "packed", 1), packed.numel(), _stream(dev)))
+    return packed
+
+
+def any4_dequant_bits(bits: int, packed: torch.Tensor, n: int, k: int, group: int,
+                      out: torch.Tensor | None = None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((n, k), dtype=torch.bfloat16, device=packed.device)
+    _check(lib.any4_dequant_bits(bits, _dev(packed, "packed", 1), n, k, group, _dev(out, "out", 2, (n, k)),
+                                 _stream(packed.device)))
+    return out
+
+
+def any4_linear_bits(bits: int, x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: int,
+                     out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = workspace_for(m, n, k, group, x.device)
+    _check(lib.any4_linear_bits(bits, _dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
+                                _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
+                                workspace.numel(), _stream(x.device)))
+    return out
 
 
 def any4_dequant(packed: torch.Tensor, n: int, k: int, group: int,

@@ -103,6 +103,53 @@ int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int 
   return e == cudaSuccess ? ANY4_OK : fail_cuda(e);
 }
 
+size_t any4_packed_bytes_bits(int bits, int n, int k, int group) {
+  if (!any4::bits_ok(bits) || !any4::shape_ok(n, k, group)) return 0;
+  return any4::make_layout(n, k, group, bits).total;
+}
+
+int any4_pack_bits(int bits, const uint8_t* idx_nib, const uint16_t* lut, const uint16_t* alpha,
+                   const uint16_t* beta, int n, int k, int group, void* packed, size_t packed_bytes,
+                   any4_stream_t stream) {
+  if (!idx_nib || !lut || !alpha || !beta || !packed) return ANY4_EINVAL;
+  if (!any4::bits_ok(bits) || !any4::shape_ok(n, k, group)) return ANY4_ESHAPE;
+  if (!aligned(packed, 16)) return ANY4_EALIGN;
+  const any4::Layout L = any4::make_layout(n, k, group, bits);
+  if (packed_bytes < L.total) return ANY4_EWORKSPACE;
+  const cudaError_t e = any4::launch_pack(idx_nib, lut, alpha, beta, L,
+                                          static_cast<uint8_t*>(packed), (cudaStream_t)stream);
+  return e == cudaSuccess ? ANY4_OK : fail_cuda(e);
+}
+
+int any4_dequant_bits(int bits, const void* packed, int n, int k, int group, uint16_t* w,
+                      any4_stream_t stream) {
+  if (!packed || !w) return ANY4_EINVAL;
+  if (!any4::bits_ok(bits) || !any4::shape_ok(n, k, group)) return ANY4_ESHAPE;
+  if (!aligned(packed, 16) || !aligned(w, 4)) return ANY4_EALIGN;
+  const any4::Layout L = any4::make_layout(n, k, group, bits);
+  const cudaError_t e = any4::launch_dequant(static_cast<const uint8_t*>(packed), L, w,
+                                             (cudaStream_t)stream);
+  return e == cudaSuccess ? ANY4_OK : fail_cuda(e);
+}
+
+int any4_linear_bits(int bits, const uint16_t* x, const void* packed, int m, int n, int k, int group,
+                     uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream) {
+  if (!x || !packed || !y || !workspace) return ANY4_EINVAL;
+  if (!any4::bits_ok(bits) || m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group))
+    return ANY4_ESHAPE;
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(y, 4) || !aligned(workspace, 16))
+    return ANY4_EALIGN;
+  int sms = 0;
+  const int st = current_sm_count(&sms);
+  if (st != ANY4_OK) return st;
+  const any4::Layout L = any4::make_layout(n, k, group, bits);
+  const any4::LinearPlan plan = any4::plan_linear(m, L, sms);
+  if (workspace_bytes < plan.workspace_bytes) return ANY4_EWORKSPACE;
+  const cudaError_t e = any4::launch_linear(x, static_cast<const uint8_t*>(packed), L, m, y,
+                                            workspace, plan, (cudaStream_t)stream);
+  return e == cudaSuccess ? ANY4_OK : fail_cuda(e);
+}
+
 const char* any4_strerror(int status) {
   switch (status) {
     case ANY4_OK: return "ANY4_OK: success";

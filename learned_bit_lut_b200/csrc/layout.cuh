@@ -32,6 +32,16 @@
 //            word 1: beta(g)    | beta(g+16)  << 16
 //            word 2: alpha(g+8) | alpha(g+24) << 16   (row pair g+8)
 //            word 3: beta(g+8)  | beta(g+24)  << 16
+//
+// any3 / any2 (b = 3, 2 bits per index; the variants named in the abstract
+// of the "any4: Learned 4-bit Numeric Representation for LLMs" summary
+// page): the same panels, chunks, lanes and steps, but a lane's 32
+// row-pair codes of a chunk (code f = 4s + q of step s; q = 0: pair g at c0,
+// 1: pair g+8 at c0, 2: pair g at c1, 3: pair g+8 at c1; a code is
+// idx(r) | idx(r+16) << b) are packed densely, code f at bit 2b*f of the
+// lane's 64b-bit string: b = 2 -> 4 words per lane, chunk [lane][4 words]
+// (512 B); b = 3 -> 6 words per lane, chunk [lane][words 0-3] then
+// [lane][words 4-5] (768 B). Weights take Np*K*b/8 bytes.
 #pragma once
 
 #include <cstddef>
@@ -50,6 +60,8 @@ constexpr int kMaxTokens = 1 << 20;     // M of any4_linear (M > 16 takes the pr
 
 struct Layout {
   int n, k, g;
+  int bits;         // bits per index: 4 (any4), 3 (any3), 2 (any2)
+  int chunk_bytes;  // 1024, 768, 512
   int n_pad;        // n rounded up to a multiple of 32
   int tiles;        // n_pad / 16
   int panels;       // n_pad / 32
@@ -67,16 +79,20 @@ inline bool shape_ok(int n, int k, int g) {
   return k % g == 0;
 }
 
-inline Layout make_layout(int n, int k, int g) {
+inline bool bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4; }
+
+inline Layout make_layout(int n, int k, int g, int bits = 4) {
   Layout L{};
   L.n = n; L.k = k; L.g = g;
+  L.bits = bits;
+  L.chunk_bytes = kChunkBytes * bits / 4;
   L.n_pad = (int)align_up((size_t)n, kPanelRows);
   L.tiles = L.n_pad / kTileRows;
   L.panels = L.n_pad / kPanelRows;
   L.kchunks = k / kChunkCols;
   L.groups = k / g;
   L.w_off = 0;
-  L.lut_off = align_up((size_t)L.n_pad * k / 2, kAlign);
+  L.lut_off = align_up((size_t)L.panels * L.kchunks * L.chunk_bytes, kAlign);
   L.ab_off = L.lut_off + align_up((size_t)L.n_pad * 32, kAlign);
   L.total = L.ab_off + align_up((size_t)L.panels * L.groups * kGroupScaleBytes, kAlign);
   return L;

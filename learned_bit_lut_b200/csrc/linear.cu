@@ -200,9 +200,27 @@ __device__ __forceinline__ void store_out(const Params& p, int P, int o, float v
   }
 }
 
-template <int MODE>
+// Shared address of the row-pair table entry for code f (= 4s + q) of a lane's
+// chunk words: 4 bits per index -> byte f of the words, dropped into address
+// bits 8..15 by one byte permute; 3 and 2 bits -> the 2b-bit code at bit
+// 2b*f of the lane's bit string, moved to bits 8.. by a (funnel) shift and
+// merged with the lane's base by one logic op.
+template <int BITS>
+__device__ __forceinline__ uint32_t pair_addr(const uint32_t (&w)[8], int f, uint32_t base) {
+  if (BITS == 4) return prmt(w[f >> 2], base, 0x7604u | ((uint32_t)(f & 3) << 4));
+  const int bit = 2 * BITS * f, word = bit >> 5, off = bit & 31;
+  uint32_t x;
+  if (off + 2 * BITS <= 32)
+    x = off >= 8 ? (w[word] >> (off - 8)) : (w[word] << (8 - off));
+  else
+    x = __funnelshift_r(w[word], w[word + 1], off - 8);
+  return (x & (((1u << (2 * BITS)) - 1u) << 8)) | base;
+}
+
+template <int MODE, int BITS>
 __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Params p) {
   using C = Cfg<MODE>;
+  constexpr int kCB = kChunkBytes * BITS / 4;   // bytes per chunk: 1024, 768, 512
   constexpr int NS = C::kNS, NF = C::kNF, NW = C::kNW, NCT = NW * 32;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
@@ -263,13 +281,13 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     while (cur.valid()) {
       const int slot = issued % NS;
       const int n = min(kPieceChunks, cur.cend - cur.c);
-      const uint32_t wbytes = (uint32_t)n * kChunkBytes;
+      const uint32_t wbytes = (uint32_t)n * kCB;
       if (issued >= NS)   // the consumer's release of the slot's previous use
         wait_bar(empty_bar(lane, slot), (uint32_t)(issued / NS - 1) & 1u, abort);
       if (*abort) break;
       const uint32_t fb = full_bar(lane, slot), dst = slot_addr(lane, slot);
       mbar_arrive_expect_tx(fb, wbytes);
-      bulk_g2s(dst, wbase + (((size_t)cur.panel * kc + cur.c) << 10), wbytes, fb);
+      bulk_g2s(dst, wbase + ((size_t)cur.panel * kc + cur.c) * kCB, wbytes, fb);
       ++issued;
       cur.c += n;
       cur.settle();
@@ -358,6 +376,23 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
   // 8*blh .. 8*blh+7; every entry goes to its four bank copies
   constexpr int kBuildPer = (512 + NCT - 1) / NCT;   // 512 tasks per panel
+  // 3- and 2-bit tables: one task per (row pair, entry), 16 << 2b tasks; the
+  // task's entry value (LUT_r[lo], LUT_r+16[hi]) is loaded a panel ahead
+  constexpr int kSmallTasks = 16 << (2 * BITS);
+  constexpr int kSmallPer = BITS == 4 ? 1 : (kSmallTasks + NCT - 1) / NCT;
+  uint32_t sv[kSmallPer], snv[kSmallPer];
+  auto load_small = [&](int P, uint32_t (&dv)[kSmallPer]) {
+#pragma unroll
+    for (int r = 0; r < kSmallPer; ++r) {
+      const int task = tid + r * NCT;
+      if (task >= kSmallTasks) break;
+      const int brp = task & 15, e = task >> 4;
+      const int br0 = (brp & 7) + 8 * (brp >> 3);
+      const int lo = e & ((1 << BITS) - 1), hi = e >> BITS;
+      const uint16_t* base_lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off) + (size_t)P * kPanelRows * 16;
+      dv[r] = ld_nc_u16(base_lut + br0 * 16 + lo) | (ld_nc_u16(base_lut + (br0 + 16) * 16 + hi) << 16);
+    }
+  };
   const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off);
   // this thread's LUT values of the panel being built (lw/lh) and of the
   // next one (nw/nh), loaded a full panel ahead
@@ -379,8 +414,13 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       }
     }
   };
-  load_lut(P0, lw, lh);
-  if (P0 < P1) load_lut(P0 + 1, nw, nh);
+  if (BITS == 4) {
+    load_lut(P0, lw, lh);
+    if (P0 < P1) load_lut(P0 + 1, nw, nh);
+  } else {
+    load_small(P0, sv);
+    if (P0 < P1) load_small(P0 + 1, snv);
+  }
 
   // lookup address bases: byte b of a word goes to address bits 8..15
   const uint32_t baseA = kTabAddr | ((uint32_t)g << 4) | ((uint32_t)t << 2);   // pairs (g, g+16)
@@ -439,10 +479,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         uint32_t a[4];
-        a[0] = lds32(prmt(w[s], baseA, 0x7604u));
-        a[1] = lds32(prmt(w[s], baseB, 0x7614u));
-        a[2] = lds32(prmt(w[s], baseA, 0x7624u));
-        a[3] = lds32(prmt(w[s], baseB, 0x7634u));
+        a[0] = lds32(pair_addr<BITS>(w, 4 * s + 0, baseA));
+        a[1] = lds32(pair_addr<BITS>(w, 4 * s + 1, baseB));
+        a[2] = lds32(pair_addr<BITS>(w, 4 * s + 2, baseA));
+        a[3] = lds32(pair_addr<BITS>(w, 4 * s + 3, baseB));
         a[0] = fma_bf16x2(a[0], sc.x, sc.y);
         a[2] = fma_bf16x2(a[2], sc.x, sc.y);
         a[1] = fma_bf16x2(a[1], sc.z, sc.w);
@@ -457,10 +497,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
         uint32_t e[2][4];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-          e[u][0] = lds32(prmt(w[s + u], baseA, 0x7604u));
-          e[u][1] = lds32(prmt(w[s + u], baseB, 0x7614u));
-          e[u][2] = lds32(prmt(w[s + u], baseA, 0x7624u));
-          e[u][3] = lds32(prmt(w[s + u], baseB, 0x7634u));
+          e[u][0] = lds32(pair_addr<BITS>(w, 4 * (s + u) + 0, baseA));
+          e[u][1] = lds32(pair_addr<BITS>(w, 4 * (s + u) + 1, baseB));
+          e[u][2] = lds32(pair_addr<BITS>(w, 4 * (s + u) + 2, baseA));
+          e[u][3] = lds32(pair_addr<BITS>(w, 4 * (s + u) + 3, baseB));
           e[u][0] = fma_bf16x2(e[u][0], sc.x, sc.y);
           e[u][2] = fma_bf16x2(e[u][2], sc.x, sc.y);
           e[u][1] = fma_bf16x2(e[u][1], sc.z, sc.w);
@@ -483,10 +523,23 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 
   for (int P = P0; P <= P1; ++P) {
     // ---- build the 16 row-pair tables of panel P
+    if (BITS != 4) {
+#pragma unroll
+      for (int r = 0; r < kSmallPer; ++r) {
+        const int task = tid + r * NCT;
+        if (task >= kSmallTasks) break;
+        const int brp = task & 15, e = task >> 4;
+        const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
+        sts128(bdst + ((uint32_t)e << 8), sv[r], sv[r], sv[r], sv[r]);
+      }
+#pragma unroll
+      for (int r = 0; r < kSmallPer; ++r) sv[r] = snv[r];
+      if (P + 1 < P1) load_small(P + 2, snv);
+    }
 #pragma unroll
     for (int r = 0; r < kBuildPer; ++r) {
       const int task = tid + r * NCT;
-      if (task >= 512) break;
+      if (BITS != 4 || task >= 512) break;
       const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
       const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
       const uint32_t L[4] = {lw[r].x, lw[r].y, lw[r].z, lw[r].w};
@@ -497,9 +550,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
         sts128(bdst + (e << 8), v, v, v, v);
       }
     }
+    if (BITS == 4) {
 #pragma unroll
-    for (int r = 0; r < kBuildPer; ++r) { lw[r] = nw[r]; lh[r] = nh[r]; }
-    if (P + 1 < P1) load_lut(P + 2, nw, nh);
+      for (int r = 0; r < kBuildPer; ++r) { lw[r] = nw[r]; lh[r] = nh[r]; }
+      if (P + 1 < P1) load_lut(P + 2, nw, nh);
+    }
     if (P == P0) {
       // activations, y and the workspace are touched only from here on
       asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -525,8 +580,15 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       wait_bar(full_bar(warp, slot), (uint32_t)(q / NS) & 1u, abort);
       ++q;
       for (int cc = 0; cc < n; ++cc) {
-        const uint4 wa = lds128(sb + (uint32_t)cc * kChunkBytes);
-        const uint4 wb = lds128(sb + (uint32_t)cc * kChunkBytes + 512u);
+        // this lane's words of the chunk: 8 (4 bits), 6 (3 bits) or 4 (2 bits)
+        const uint4 wa = lds128(sb + (uint32_t)cc * kCB);
+        uint4 wb = make_uint4(0u, 0u, 0u, 0u);
+        if (BITS == 4) wb = lds128(sb + (uint32_t)cc * kCB + 512u);
+        if (BITS == 3) {
+          const uint2 w2 = lds64(sb - 8u * lane + (uint32_t)cc * kCB + 512u);
+          wb.x = w2.x;
+          wb.y = w2.y;
+        }
         // release the slot once its last words are in registers
         if (cc == n - 1) mbar_arrive_after(empty_bar(warp, slot), wa.x, wb.x, 0u, 0u);
         uint32_t xw[NX][8];
@@ -556,10 +618,18 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   if (tid == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
 }
 
-template <int MODE>
+template <int MODE, int BITS>
 cudaError_t allow_smem_mode() {
-  return cudaFuncSetAttribute(linear_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(linear_kernel<MODE, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               Cfg<MODE>::kSmemBytes);
+}
+
+template <int BITS>
+cudaError_t allow_smem_bits() {
+  cudaError_t e = allow_smem_mode<0, BITS>();
+  if (e == cudaSuccess) e = allow_smem_mode<1, BITS>();
+  if (e == cudaSuccess) e = allow_smem_mode<2, BITS>();
+  return e;
 }
 
 cudaError_t allow_large_smem() {
@@ -569,14 +639,14 @@ cudaError_t allow_large_smem() {
   if (e != cudaSuccess) return e;
   const unsigned long long bit = 1ull << (dev & 63);
   if (done_mask.load(std::memory_order_relaxed) & bit) return cudaSuccess;
-  e = allow_smem_mode<0>();
-  if (e == cudaSuccess) e = allow_smem_mode<1>();
-  if (e == cudaSuccess) e = allow_smem_mode<2>();
+  e = allow_smem_bits<4>();
+  if (e == cudaSuccess) e = allow_smem_bits<3>();
+  if (e == cudaSuccess) e = allow_smem_bits<2>();
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_relaxed);
   return e;
 }
 
-template <int MODE>
+template <int MODE, int BITS>
 cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t stream) {
   // programmatic dependent launch: this kernel's weight prologue may overlap the
   // tail of the previous kernel on the stream (see griddepcontrol in the kernel)
@@ -590,7 +660,16 @@ cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t st
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, linear_kernel<MODE>, p);
+  return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS>, p);
+}
+
+template <int BITS>
+cudaError_t launch_bits(const Params& p, const LinearPlan& plan, cudaStream_t stream) {
+  switch (plan.mode) {
+    case 0: return launch_mode<0, BITS>(p, plan, stream);
+    case 1: return launch_mode<1, BITS>(p, plan, stream);
+    default: return launch_mode<2, BITS>(p, plan, stream);
+  }
 }
 
 }  // namespace
@@ -636,10 +715,10 @@ cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout
   p.ctas = plan.ctas;
   p.units = plan.units;
   p.w_off = L.w_off; p.lut_off = L.lut_off; p.ab_off = L.ab_off;
-  switch (plan.mode) {
-    case 0: return launch_mode<0>(p, plan, stream);
-    case 1: return launch_mode<1>(p, plan, stream);
-    default: return launch_mode<2>(p, plan, stream);
+  switch (L.bits) {
+    case 3: return launch_bits<3>(p, plan, stream);
+    case 2: return launch_bits<2>(p, plan, stream);
+    default: return launch_bits<4>(p, plan, stream);
   }
 }
 

@@ -60,6 +60,46 @@ __global__ void pack_weights_kernel(const uint8_t* __restrict__ idx_nib, Layout 
   }
 }
 
+// b-bit weights (b = 2, 3; layout.cuh): one thread per (panel, chunk, lane)
+// builds the lane's 32 row-pair codes and writes its 2b packed words.
+template <int B>
+__global__ void pack_weights_bits_kernel(const uint8_t* __restrict__ idx_nib, Layout L,
+                                         uint32_t* __restrict__ out) {
+  constexpr int W = 2 * B;
+  constexpr uint32_t mask = (1u << B) - 1u;
+  const size_t total = (size_t)L.panels * L.kchunks * 32;
+  const size_t row_bytes = (size_t)L.k / 2;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const int lane = (int)(e & 31);
+    const size_t pc = e >> 5;
+    const int chunk = (int)(pc % L.kchunks);
+    const size_t panel = pc / L.kchunks;
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t wd[W];
+    for (int j = 0; j < W; ++j) wd[j] = 0u;
+    for (int f = 0; f < 32; ++f) {
+      const int st = f >> 2, q = f & 3;
+      const int col = chunk * kChunkCols + 16 * t + 2 * st + (q >> 1);
+      uint32_t code = 0;
+      for (int u = 0; u < 2; ++u) {
+        const size_t row = panel * kPanelRows + g + 8 * (q & 1) + 16 * u;
+        if (row >= (size_t)L.n) continue;
+        const uint32_t nib = (idx_nib[row * row_bytes + col / 2] >> (4 * (col & 1))) & mask;
+        code |= nib << (B * u);
+      }
+      const int bit = 2 * B * f, word = bit >> 5, off = bit & 31;
+      wd[word] |= code << off;
+      if (off + 2 * B > 32) wd[word + 1] |= code >> (32 - off);
+    }
+    const size_t base = (panel * L.kchunks + chunk) * (size_t)L.chunk_bytes / 4;
+    for (int j = 0; j < W; ++j) {
+      const size_t at = j < 4 ? base + (size_t)lane * 4 + j : base + 128 + (size_t)lane * (W - 4) + (j - 4);
+      out[at] = wd[j];
+    }
+  }
+}
+
 __global__ void pack_lut_kernel(const uint16_t* __restrict__ lut, Layout L,
                                 uint16_t* __restrict__ out) {
   const size_t total = (size_t)L.n_pad * 16;
@@ -131,6 +171,48 @@ __global__ void dequant_kernel(const uint8_t* __restrict__ packed, Layout L,
         const float v = fmaf(a, bf16_bits_to_float(lutsec[row * 16 + idx]), c);   // one fp32 rounding
         const __nv_bfloat16 h = __float2bfloat16_rn(v);                            // then bf16
         w[row * L.k + col] = *reinterpret_cast<const uint16_t*>(&h);
+      }
+    }
+  }
+}
+
+// b-bit dequant (b = 2, 3): one thread per (panel, chunk, lane); same
+// arithmetic as dequant_kernel.
+template <int B>
+__global__ void dequant_bits_kernel(const uint8_t* __restrict__ packed, Layout L, uint16_t* __restrict__ w) {
+  constexpr int W = 2 * B;
+  constexpr uint32_t mask = (1u << B) - 1u;
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(packed + L.w_off);
+  const uint16_t* lutsec = reinterpret_cast<const uint16_t*>(packed + L.lut_off);
+  const uint32_t* ab = reinterpret_cast<const uint32_t*>(packed + L.ab_off);
+  const size_t total = (size_t)L.panels * L.kchunks * 32;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const int lane = (int)(e & 31);
+    const size_t pc = e >> 5;
+    const int chunk = (int)(pc % L.kchunks);
+    const size_t panel = pc / L.kchunks;
+    const int g = lane >> 2, t = lane & 3;
+    const size_t base = (panel * L.kchunks + chunk) * (size_t)L.chunk_bytes / 4;
+    uint32_t wd[W + 1];
+    for (int j = 0; j < W; ++j)
+      wd[j] = words[j < 4 ? base + (size_t)lane * 4 + j : base + 128 + (size_t)lane * (W - 4) + (j - 4)];
+    wd[W] = 0u;
+    for (int f = 0; f < 32; ++f) {
+      const int st = f >> 2, q = f & 3;
+      const int col = chunk * kChunkCols + 16 * t + 2 * st + (q >> 1);
+      const int bit = 2 * B * f, word = bit >> 5, off = bit & 31;
+      const uint32_t code = (uint32_t)((((uint64_t)wd[word + 1] << 32) | wd[word]) >> off);
+      const uint32_t* sc = ab + ((panel * L.groups + col / L.g) * 8 + g) * 4 + 2 * (q & 1);
+      for (int u = 0; u < 2; ++u) {
+        const size_t row = panel * kPanelRows + g + 8 * (q & 1) + 16 * u;
+        if (row >= (size_t)L.n) continue;
+        const uint32_t idx = (code >> (B * u)) & mask;
+        const float a = bf16_bits_to_float((sc[0] >> (16 * u)) & 0xFFFFu);
+        const float c = bf16_bits_to_float((sc[1] >> (16 * u)) & 0xFFFFu);
+        const float v = fmaf(a, bf16_bits_to_float(lutsec[row * 16 + idx]), c);
+        const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+        w[row * L.k + col] = *reinterpret_cast<const uint16_t*>(&hv);
       }
     }
   }
@@ -210,12 +292,23 @@ static int grid_for(size_t work, int threads) {
   return (int)(b ? b : 1);
 }
 
+static void launch_pack_weights(const uint8_t* idx_nib, const Layout& L, uint8_t* packed, cudaStream_t stream) {
+  const int th = 256;
+  uint32_t* out = reinterpret_cast<uint32_t*>(packed + L.w_off);
+  const size_t lanes = (size_t)L.panels * L.kchunks * 32;
+  if (L.bits == 3)
+    pack_weights_bits_kernel<3><<<grid_for(lanes, th), th, 0, stream>>>(idx_nib, L, out);
+  else if (L.bits == 2)
+    pack_weights_bits_kernel<2><<<grid_for(lanes, th), th, 0, stream>>>(idx_nib, L, out);
+  else
+    pack_weights_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(idx_nib, L, out);
+}
+
 cudaError_t launch_pack(const uint8_t* idx_nib, const uint16_t* lut, const uint16_t* alpha,
                         const uint16_t* beta, const Layout& L, uint8_t* packed,
                         cudaStream_t stream) {
   const int th = 256;
-  pack_weights_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(
-      idx_nib, L, reinterpret_cast<uint32_t*>(packed + L.w_off));
+  launch_pack_weights(idx_nib, L, packed, stream);
   pack_lut_kernel<<<grid_for((size_t)L.n_pad * 16, th), th, 0, stream>>>(
       lut, L, reinterpret_cast<uint16_t*>(packed + L.lut_off));
   pack_scales_kernel<<<grid_for((L.total - L.ab_off) / 4, th), th, 0, stream>>>(
@@ -229,8 +322,7 @@ cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
   const int th = 256;
   Table16 t;
   for (int q = 0; q < 16; ++q) t.v[q] = lut[q];
-  pack_weights_kernel<<<grid_for((size_t)L.n_pad * L.k / 8, th), th, 0, stream>>>(
-      idx_nib, L, reinterpret_cast<uint32_t*>(packed + L.w_off));
+  launch_pack_weights(idx_nib, L, packed, stream);
   pack_lut_fixed_kernel<<<grid_for((size_t)L.n_pad * 16, th), th, 0, stream>>>(
       t, L, reinterpret_cast<uint16_t*>(packed + L.lut_off));
   pack_scales_kernel<<<grid_for((L.total - L.ab_off) / 4, th), th, 0, stream>>>(
@@ -241,7 +333,12 @@ cudaError_t launch_pack_fixed(const uint8_t* idx_nib, const uint16_t (&lut)[16],
 cudaError_t launch_dequant(const uint8_t* packed, const Layout& L, uint16_t* w,
                            cudaStream_t stream) {
   const int th = 256;
-  if ((reinterpret_cast<uintptr_t>(w) & 15) == 0) {   // 16-byte stores need a 16-byte aligned w
+  const size_t lanes = (size_t)L.panels * L.kchunks * 32;
+  if (L.bits == 3) {
+    dequant_bits_kernel<3><<<grid_for(lanes, th), th, 0, stream>>>(packed, L, w);
+  } else if (L.bits == 2) {
+    dequant_bits_kernel<2><<<grid_for(lanes, th), th, 0, stream>>>(packed, L, w);
+  } else if ((reinterpret_cast<uintptr_t>(w) & 15) == 0) {   // 16-byte stores need a 16-byte aligned w
     const dim3 grid((L.kchunks + kDqChunks - 1) / kDqChunks, L.panels);
     dequant_tile_kernel<<<grid, th, 0, stream>>>(packed, L, w);
   } else {

@@ -109,3 +109,20 @@ def test_quantize_rejects_bad_arguments():
     assert q(d, d, 32, 64, 64, 4, -1, d, d, d, d, None) == a4.ANY4_EINVAL      # iters
     assert q(d, d, 31, 64, 64, 4, 10, d, d, d, d, None) == a4.ANY4_ESHAPE
     assert q(d, d, 32, 64, 96, 4, 10, d, d, d, d, None) == a4.ANY4_ESHAPE
+
+
+def test_bits_sizes_and_rejection():
+    # dense any3 / any2 packing: N_pad*K*b/8 bytes of indices, same LUT and scales
+    n, k, g = 4096, 4096, 128
+    lut, ab = 32 * n, 4 * n * (k // g)
+    assert a4.any4_packed_bytes_bits(4, n, k, g) == a4.any4_packed_bytes(n, k, g)
+    assert a4.any4_packed_bytes_bits(3, n, k, g) == n * k * 3 // 8 + lut + ab
+    assert a4.any4_packed_bytes_bits(2, n, k, g) == n * k // 4 + lut + ab
+    for bad in (0, 1, 5, 8, -3):
+        assert a4.any4_packed_bytes_bits(bad, n, k, g) == 0
+    p = ctypes.c_void_p(256)
+    assert a4.lib.any4_pack_bits(5, p, p, p, p, 64, 64, 64, p, 1 << 30, None) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_dequant_bits(1, p, 64, 64, 64, p, None) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_bits(6, p, p, 1, 64, 64, 64, p, p, 1 << 30, None) == a4.ANY4_ESHAPE
+    z = ctypes.c_void_p(0)
+    assert a4.lib.any4_pack_bits(3, z, p, p, p, 64, 64, 64, p, 1 << 30, None) == a4.ANY4_EINVAL

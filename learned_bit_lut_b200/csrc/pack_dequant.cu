@@ -242,14 +242,17 @@ __global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __rest
   const int i = wi & 3, ln = (wi >> 2) & 31, h = wi >> 7;
   const int g = ln >> 2, t = ln & 3;
   const int c0 = 16 * t + 2 * (4 * h + i);   // column within a chunk
+  const int gshift = __ffs(L.g) - 1;         // G is a power of two
+  const uint32_t* wsrc = words + ((size_t)P * L.kchunks + c_begin) * 256 + wi;
+  const uint4* ssrc = reinterpret_cast<const uint4*>(ab) + (size_t)P * L.groups * 8 + g;
   uint32_t word[kDqChunks];
   uint4 sc[kDqChunks];
 #pragma unroll
   for (int j = 0; j < kDqChunks; ++j) {
     if (j < nch) {
       const int col0 = (c_begin + j) * kChunkCols + c0;
-      word[j] = __ldg(words + ((size_t)P * L.kchunks + c_begin + j) * 256 + wi);
-      sc[j] = __ldg(reinterpret_cast<const uint4*>(ab + (((size_t)P * L.groups + col0 / L.g) * 8 + g) * 4));
+      word[j] = __ldg(wsrc + j * 256);
+      sc[j] = __ldg(ssrc + (size_t)(col0 >> gshift) * 8);
     }
   }
   for (int e = threadIdx.x; e < kPanelRows * 16; e += blockDim.x)
@@ -276,13 +279,23 @@ __global__ void __launch_bounds__(256) dequant_tile_kernel(const uint8_t* __rest
     }
   }
   __syncthreads();
-  const int units = nch * kChunkCols / 8;   // 16-byte units per row
-  for (int e = threadIdx.x; e < kPanelRows * units; e += blockDim.x) {
-    const int r = e / units, u = e % units;
-    const size_t row = (size_t)P * kPanelRows + r;
-    if (row >= (size_t)L.n) continue;
-    const uint4 v = *reinterpret_cast<const uint4*>(&tile[r * kDqRow + u * 8]);
-    *reinterpret_cast<uint4*>(w + row * L.k + (size_t)c_begin * kChunkCols + u * 8) = v;
+  uint16_t* wp = w + (size_t)P * kPanelRows * L.k + (size_t)c_begin * kChunkCols;
+  const int rows = min(kPanelRows, L.n - P * kPanelRows);
+  if (nch == kDqChunks) {   // full strip: 64 16-byte units per row, 4 rows per pass
+    const int u = threadIdx.x & 63;
+#pragma unroll
+    for (int r = threadIdx.x >> 6; r < kPanelRows; r += 4)
+      if (r < rows)
+        *reinterpret_cast<uint4*>(wp + (size_t)r * L.k + u * 8) =
+            *reinterpret_cast<const uint4*>(&tile[r * kDqRow + u * 8]);
+  } else {
+    const int units = nch * kChunkCols / 8;   // 16-byte units per row
+    for (int e = threadIdx.x; e < kPanelRows * units; e += blockDim.x) {
+      const int r = e / units, u = e % units;
+      if (r < rows)
+        *reinterpret_cast<uint4*>(wp + (size_t)r * L.k + u * 8) =
+            *reinterpret_cast<const uint4*>(&tile[r * kDqRow + u * 8]);
+    }
   }
 }
 

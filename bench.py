@@ -143,6 +143,49 @@ def cpu_baseline(budget_s: float, calls=None):
                       f"fp64 matmul ({blas} BLAS threads)"}
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time (all ranks take part; NCCL on GPUs, gloo on CPU)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes: int, n_calls: int,
+                per_m: dict, peak: float, peak_kind: str, clocks, e2e, cpu) -> dict:
+    """The JSON line of one run: whole-job throughput over all ranks (weak
+    scaling: every rank runs the full step) and the roofline of the kernel."""
+    achieved = step_bytes / (ms_step * 1e6)
+    return {
+        "metric": "any4_linear achieved HBM GB/s (algorithmic bytes)",
+        "value": step_bytes * world / (ms_step * 1e6), "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS,
+                   "linears_per_layer": len(synth.LLAMA3_8B_LAYER), "ms": list(MS),
+                   "group": GROUP, "calls_per_step": n_calls,
+                   "l2": "inputs larger than L2: 3.76 GB of distinct packed weights per step",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_call": ms_step * 1e3 / n_calls,
+        "by_m": per_m,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak,
+                     "traffic": (DRAM_PER_ALGO_BYTE * step_bytes / n_calls
+                                 if DRAM_PER_ALGO_BYTE is not None else None),
+                     "traffic_note": "dram bytes per launch: ncu dram__bytes_read+write of one "
+                                     "14336x4096 M=1 launch over its algorithmic bytes, times "
+                                     "this step's mean algorithmic bytes per launch",
+                     "peak_source": f"{peak_kind} hbm_gbs", "kernel": "linear_kernel"},
+        "gpu_launches": n_calls * steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+
+
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
@@ -236,12 +279,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             fn()
         e1.record()
         barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     def step():
         for mm in MS:
@@ -263,9 +301,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         per_m[str(mm)] = {"us_per_call": ms_m * 1e3 / len(sel[mm]), "GB/s": b / (ms_m * 1e6)}
 
     step_bytes = sum(algorithmic_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
-    value = step_bytes * world / (ms_step * 1e6)
     peak, peak_kind = read_peaks()
-    achieved = step_bytes / (ms_step * 1e6)
 
     # end to end through the Python API: pinned host x in, y out, every step
     e2e = None
@@ -296,31 +332,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         cpu = cpu_baseline(args.cpu_seconds)
 
     if rank == 0:
-        line = {
-            "metric": "any4_linear achieved HBM GB/s (algorithmic bytes)",
-            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS,
-                       "linears_per_layer": len(synth.LLAMA3_8B_LAYER), "ms": list(MS),
-                       "group": GROUP, "calls_per_step": len(calls),
-                       "l2": "inputs larger than L2: 3.76 GB of distinct packed weights per step",
-                       "parallelism": f"replicas x{world}"},
-            "us_per_call": ms_step * 1e3 / len(calls),
-            "by_m": per_m,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak,
-                         "traffic": (DRAM_PER_ALGO_BYTE * step_bytes / len(calls)
-                                     if DRAM_PER_ALGO_BYTE is not None else None),
-                         "traffic_note": "dram bytes per launch: ncu dram__bytes_read+write of one "
-                                         "14336x4096 M=1 launch over its algorithmic bytes, times "
-                                         "this step's mean algorithmic bytes per launch",
-                         "peak_source": f"{peak_kind} hbm_gbs", "kernel": "linear_kernel"},
-            "gpu_launches": len(calls) * args.steps,
-            "clocks": sampler.summary(),
-            "e2e": e2e,
-            "cpu_baseline": cpu,
-        }
+        line = result_line(world, args.steps, args.warmup, ms_step, step_bytes, len(calls), per_m,
+                           peak, peak_kind, sampler.summary(), e2e, cpu)
         print(json.dumps(line), flush=True)
     for g in graphs.values():
         del g

@@ -678,7 +678,7 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   LinearPlan pl{};
   if (m > 16) {   // prefill: dequantized W scratch + tensor-core GEMM
     pl.mode = 3;
-    pl.workspace_bytes = prefill_workspace_bytes(L);
+    pl.workspace_bytes = prefill_workspace_bytes(L, m, num_sms);
     pl.ctas = num_sms;
     return pl;
   }

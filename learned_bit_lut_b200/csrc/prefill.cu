@@ -10,7 +10,11 @@
 //      tensor memory) += W_hat tile (128 x 64, shared memory) . x tile^T
 //      (256 x 64, shared memory), both operands brought in by TMA with the
 //      128-byte swizzle, 4 pipeline stages, two accumulators so the epilogue
-//      of one tile overlaps the main loop of the next.
+//      of one tile overlaps the main loop of the next. When there are fewer
+//      output tiles than SMs, each tile's K range is split between up to
+//      SMs/tiles blocks (split-K): they store fp32 partials in the workspace
+//      and the last one to arrive adds them in split order (deterministic)
+//      and writes y.
 // Dequantizing on the fly into shared memory instead would cost about two
 // instructions per weight on B200 (lookup, scale, store), while tensor memory
 // holds at most 512 tokens of fp32 accumulators per 128 rows: the decode
@@ -59,7 +63,17 @@ struct GemmCtl {
   uint64_t acc_empty[2];
   uint32_t tmem_base;
   int abort_flag;
+  int last_split;   // epilogue: this block finishes the tile's split-K sum
 };
+
+constexpr int kEpilogueBar = 1;                 // named barrier of the 4 epilogue warps
+constexpr int kPartialFloats = kBM * kBN;       // one split's fp32 tile [token][row]
+constexpr int kMinSplitChunks = 8;              // K per split >= 8 stages (512 columns)
+constexpr int kMaxSplits = 4;                   // the last block reads all splits' partials
+
+__device__ __forceinline__ void epilogue_sync() {
+  asm volatile("bar.sync %0, 128;" ::"n"(kEpilogueBar) : "memory");
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -141,7 +155,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     prefill_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap,
-                        uint16_t* __restrict__ y, int m, int n, int k, unsigned* status) {
+                        uint16_t* __restrict__ y, int m, int n, int k, int splits, float* __restrict__ partials,
+                        unsigned* counters, unsigned* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_addr(smem_raw);
@@ -153,6 +168,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int n_tiles = (n + kBM - 1) / kBM, m_tiles = (m + kBN - 1) / kBN;
   const int tiles = n_tiles * m_tiles, kch = k / kBK;
+  const int units = tiles * splits;   // unit u: tile u / splits, K split u % splits
+  auto k_range = [&](int u, int& kc0, int& kc1) {
+    const int sp = u % splits;
+    kc0 = (int)((long long)sp * kch / splits);
+    kc1 = (int)((long long)(sp + 1) * kch / splits);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -183,9 +204,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------- TMA producer
     if (lane == 0) {
       int it = 0;
-      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x) {
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const int tile = u / splits;
         const int nt = tile / m_tiles, mt = tile % m_tiles;
-        for (int kc = 0; kc < kch; ++kc, ++it) {
+        int kc0, kc1;
+        k_range(u, kc0, kc1);
+        for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (it >= kStages &&
@@ -202,14 +226,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < tiles && !*abort_flag; tile += gridDim.x, ++tcount) {
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x, ++tcount) {
         const int b = tcount & 1;
         const uint32_t aph = (uint32_t)(tcount >> 1) & 1u;
         if (tcount >= 2 && !gemm_wait(smem_addr(&ctl->acc_empty[b]), aph ^ 1u, abort_flag, status))
           break;
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)b * kAccCols;
-        for (int kc = 0; kc < kch; ++kc, ++it) {
+        int kc0, kc1;
+        k_range(u, kc0, kc1);
+        for (int kc = kc0; kc < kc1; ++kc, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (uint32_t)(it / kStages) & 1u;
           if (!gemm_wait(smem_addr(&ctl->full[s]), ph, abort_flag, status)) break;
@@ -217,7 +243,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t ad = sw128_desc(sa(s)), bd = sw128_desc(sb(s));
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk)   // 16 columns = 32 bytes = 2 descriptor units
-            tc_mma(d, ad + 2u * (uint64_t)kk, bd + 2u * (uint64_t)kk, (kc | kk) != 0 ? 1u : 0u);
+            tc_mma(d, ad + 2u * (uint64_t)kk, bd + 2u * (uint64_t)kk, (kc > kc0 || kk > 0) ? 1u : 0u);
           tc_commit(smem_addr(&ctl->empty[s]));   // the stage is free once these MMAs are done
         }
         tc_commit(smem_addr(&ctl->acc_full[b]));
@@ -227,21 +253,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ---------------------------------------------------------- epilogue
     const int q = warp & 3;   // tensor-memory lane quarter of this warp
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++tcount) {
+      const int tile = u / splits;
       const int nt = tile / m_tiles, mt = tile % m_tiles;
       const int b = tcount & 1;
       const uint32_t ph = (uint32_t)(tcount >> 1) & 1u;
-      if (!gemm_wait(smem_addr(&ctl->acc_full[b]), ph, abort_flag, status)) break;
+      gemm_wait(smem_addr(&ctl->acc_full[b]), ph, abort_flag, status);
+      epilogue_sync();          // all four warps leave together if any wait gave up
+      if (*abort_flag) break;
       tc_fence_after();
-      const int row = nt * kBM + 32 * q + lane;
+      const int r = 32 * q + lane, row = nt * kBM + r;
       const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)b * kAccCols;
+      float* part = partials + (size_t)u * kPartialFloats;   // [token][row] of this split
 #pragma unroll 1
       for (int j = 0; j < kBN / 32; ++j) {
         uint32_t v[32];
         tc_ld_x32(tbase + 32u * (uint32_t)j, v);
         tc_wait_ld();
         const int m0 = mt * kBN + 32 * j;
-        if (row < n) {
+        if (splits > 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) __stcg(part + (32 * j + i) * kBM + r, __uint_as_float(v[i]));
+        } else if (row < n) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             if (m0 + i < m) {
@@ -254,6 +287,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_one(smem_addr(&ctl->acc_empty[b]));
+      if (splits > 1) {
+        // publish this split; the last of the tile's splits adds them in order
+        __threadfence();
+        epilogue_sync();
+        if (q == 0 && lane == 0) ctl->last_split = atomicAdd(counters + tile, 1u) == (unsigned)(splits - 1);
+        epilogue_sync();
+        if (ctl->last_split) {
+          __threadfence();
+          const float* base = partials + (size_t)tile * splits * kPartialFloats;
+          if (row < n) {
+            // 32 tokens at a time, so 32 loads of each split are in flight together
+#pragma unroll 1
+            for (int j0 = 0; j0 < kBN && mt * kBN + j0 < m; j0 += 32) {
+              float acc[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+#pragma unroll 1
+              for (int sp = 0; sp < splits; ++sp) {
+                const float* src = base + (size_t)sp * kPartialFloats + j0 * kBM + r;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) acc[i] += __ldcg(src + i * kBM);
+              }
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int mm = mt * kBN + j0 + i;
+                if (mm < m) {
+                  const __nv_bfloat16 h = __float2bfloat16_rn(acc[i]);
+                  y[(size_t)mm * n + row] = *reinterpret_cast<const uint16_t*>(&h);
+                }
+              }
+            }
+          }
+          epilogue_sync();
+          if (q == 0 && lane == 0) counters[tile] = 0u;   // ready for the next call
+        }
+      }
     }
   }
   tc_fence_before();
@@ -307,8 +376,25 @@ cudaError_t allow_gemm_smem() {
 
 size_t prefill_scratch_offset() { return kHeaderBytes; }
 
-size_t prefill_workspace_bytes(const Layout& L) {
+int prefill_splits(const Layout& L, int m, int num_sms) {
+  const int tiles = ((L.n + kBM - 1) / kBM) * ((m + kBN - 1) / kBN);
+  const int kch = L.k / kBK;
+  int s = tiles < num_sms ? num_sms / tiles : 1;
+  const int smax = kch / kMinSplitChunks > 0 ? kch / kMinSplitChunks : 1;
+  if (s > smax) s = smax;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s < 1 ? 1 : s;
+}
+
+size_t prefill_partials_offset(const Layout& L) {
   return kHeaderBytes + align_up((size_t)L.n * L.k * 2, kAlign);
+}
+
+size_t prefill_workspace_bytes(const Layout& L, int m, int num_sms) {
+  const int splits = prefill_splits(L, m, num_sms);
+  const int tiles = ((L.n + kBM - 1) / kBM) * ((m + kBN - 1) / kBN);
+  const size_t partials = splits > 1 ? (size_t)tiles * splits * kPartialFloats * sizeof(float) : 0;
+  return prefill_partials_offset(L) + partials;
 }
 
 cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
@@ -323,8 +409,12 @@ cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layou
   if (!encode_bf16_map(&wmap, what, L.n, L.k, kBM) || !encode_bf16_map(&xmap, x, m, L.k, kBN))
     return cudaErrorInvalidValue;
   const int tiles = ((L.n + kBM - 1) / kBM) * ((m + kBN - 1) / kBN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  const int splits = prefill_splits(L, m, num_sms);
+  const int units = tiles * splits;
+  const int grid = units < num_sms ? units : num_sms;
   unsigned* status = reinterpret_cast<unsigned*>(ws + kCountersBytes);
+  unsigned* counters = reinterpret_cast<unsigned*>(ws);
+  float* partials = reinterpret_cast<float*>(ws + prefill_partials_offset(L));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kGemmThreads);
@@ -335,7 +425,8 @@ cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layou
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, wmap, xmap, y, m, L.n, L.k, status);
+  return cudaLaunchKernelEx(&cfg, prefill_gemm_kernel, wmap, xmap, y, m, L.n, L.k, splits, partials, counters,
+                            status);
 }
 
 }  // namespace any4

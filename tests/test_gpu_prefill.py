@@ -86,3 +86,21 @@ def test_prefill_workspace_size():
     rc = a4.lib.any4_linear(x.data_ptr(), packed.data_ptr(), 17, n, k, g, y.data_ptr(), ws.data_ptr(),
                             ws.numel(), None)
     assert rc == a4.ANY4_EWORKSPACE
+
+
+@pytest.mark.parametrize("n,k,g,m", [(1024, 4096, 128, 64), (4096, 4096, 128, 17), (256, 512, 128, 300),
+                                     (1024, 1024, 64, 40)])
+def test_prefill_split_k(n, k, g, m):
+    # few output tiles: the K range of each tile is split between blocks and
+    # the partials are added in split order; two calls must agree bit for bit
+    q, s = quantized(n, k, g, layer=f"psplit{n}x{k}", iters=4)
+    x = bf16_dev(synth.activations_bf16(m, s, 11, layer=f"psplit{n}x{k}"))
+    packed = pack_dev(q)
+    ws = a4.workspace_for(m, n, k, g, torch.device("cuda:0"))
+    y1 = a4.any4_linear(x, packed, n, k, g, workspace=ws)
+    y2 = a4.any4_linear(x, packed, n, k, g, workspace=ws)
+    torch.cuda.synchronize()
+    check_linear(y1, bits_host(x), q)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert int(ws[STATUS_OFFSET:STATUS_OFFSET + 4].view(torch.int32)[0]) == 0
+    assert int(ws[:4 * 65536].view(torch.int32).abs().sum()) == 0   # tile counters back to zero

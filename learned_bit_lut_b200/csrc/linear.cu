@@ -29,15 +29,27 @@
 //    16-row tiles, which keeps one MMA per 8 tokens.
 //  * Work split: a thread block (one per SM) owns a contiguous range of
 //    (32-row panel, 64-column chunk) units (stream-K). For each panel its
-//    consumer warps build the 16 row-pair tables (64 KB) once, then split the
-//    panel's chunks. A producer warp streams every consumer warp's weights,
-//    four chunks (4 KB) per bulk copy, into per-warp rings of full/empty
-//    mbarriers; the consumers load their activation columns and alpha/beta
-//    straight from L2 (three 128-bit loads per chunk, one chunk ahead). No
-//    block-wide barrier inside a panel. The warps' fp32 tiles are summed in warp order; a panel
-//    split between thread blocks is finished by the last one to arrive, which
-//    sums the partials in thread-block order (deterministic; nothing waits on
-//    another thread block).
+//    consumer warps (16 for M <= 4, 12 for M <= 8, 8 for M <= 16: what the
+//    register file and shared memory hold) build the 16 row-pair tables
+//    (64 KB) once, then split the panel's chunks. A producer warp streams
+//    every consumer warp's weights, four chunks (4 KB) per bulk copy, into
+//    per-warp rings of full/empty mbarriers. Each consumer loads its
+//    activation columns per chunk, one chunk ahead (for M <= 8 kept in L1
+//    with evict_last), and alpha/beta per group (for M <= 8 once per group,
+//    past L1). No block-wide barrier inside a panel.
+//  * Reduction: a reducer warp sums the consumer warps' fp32 tiles in warp
+//    order. A panel split between thread blocks is finished by the block
+//    that holds its first unit, which processes it last: it waits (bounded)
+//    for the other blocks' partials, published with a release increment when
+//    they processed the panel first, and adds them in thread-block order, so
+//    results are deterministic.
+//  * The SM's shared-memory/L1 data pipe (one 128-byte wavefront per clock)
+//    bounds this decode: per chunk of a panel the lookups take 32 wavefronts,
+//    the weight words about 17 (bulk-copy write plus read), the table build 8
+//    at K = 4096, activation and alpha/beta loads the rest.
+//  * any3 / any2 (BITS = 3, 2): the same kernel with a lane's row-pair codes
+//    packed densely (layout.cuh); a code becomes a table address with a
+//    funnel shift and one logic op, and the tables have 64 / 16 entries.
 #include <cuda_bf16.h>
 
 #include <atomic>

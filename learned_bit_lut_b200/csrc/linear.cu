@@ -697,8 +697,16 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   pl.mode = m <= 4 ? 0 : m <= 8 ? 1 : 2;
   pl.nf = pl.mode == 0 ? 4 : pl.mode == 1 ? 8 : 16;
   pl.units = (long long)L.panels * L.kchunks;
-  long long c = pl.units / kMinUnitsPerCta;
-  if (c > num_sms) c = num_sms;
+  long long c;
+  if (L.panels <= num_sms) {
+    // one whole panel per thread block: no table built for a piece of a
+    // panel and no split panel to finish (on B200 this is 1.3-1.5x faster
+    // than spreading 128 panels over 148 blocks)
+    c = L.panels;
+  } else {
+    c = pl.units / kMinUnitsPerCta;
+    if (c > num_sms) c = num_sms;
+  }
   if (c < 1) c = 1;
   pl.ctas = (int)c;
   pl.partials_bytes = (size_t)pl.ctas * 32 * pl.nf * sizeof(float);

@@ -139,6 +139,8 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
 
 // Thread block whose unit range [floor(c*U/C), floor((c+1)*U/C)) holds unit u.
 __device__ __forceinline__ int cta_of_unit(long long u, long long U, int C) {
+  if ((unsigned long long)U * (unsigned)C < (1ull << 32))
+    return (int)(((unsigned)(u + 1) * (unsigned)C - 1u) / (unsigned)U);
   return (int)(((u + 1) * (long long)C - 1) / U);
 }
 
@@ -261,9 +263,24 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 
   const long long U = p.units;
   const int kc = p.kc;
-  const long long u_lo = (long long)blockIdx.x * U / p.ctas;
-  const long long u_hi = (long long)(blockIdx.x + 1) * U / p.ctas;
-  const int P0 = (int)(u_lo / kc), P1 = (int)((u_hi - 1) / kc);
+  // this block's units [u_lo, u_hi) and panels P0..P1; in 32-bit arithmetic
+  // whenever it cannot overflow (a 64-bit division costs ~300 cycles, on the
+  // critical path of every call)
+  long long u_lo, u_hi;
+  int P0, P1;
+  if ((unsigned long long)U * (unsigned)p.ctas < (1ull << 32)) {
+    const unsigned uu = (unsigned)U, nc = (unsigned)p.ctas, b = blockIdx.x;
+    const unsigned lo = b * uu / nc, hi = (b + 1) * uu / nc;
+    u_lo = lo;
+    u_hi = hi;
+    P0 = (int)(lo / (unsigned)kc);
+    P1 = (int)((hi - 1) / (unsigned)kc);
+  } else {
+    u_lo = (long long)blockIdx.x * U / p.ctas;
+    u_hi = (long long)(blockIdx.x + 1) * U / p.ctas;
+    P0 = (int)(u_lo / kc);
+    P1 = (int)((u_hi - 1) / kc);
+  }
   auto is_split = [&](int P) {
     const long long pu = (long long)P * kc;
     return !(pu >= u_lo && pu + kc <= u_hi);

@@ -268,7 +268,11 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   // critical path of every call)
   long long u_lo, u_hi;
   int P0, P1;
-  if ((unsigned long long)U * (unsigned)p.ctas < (1ull << 32)) {
+  if ((long long)p.ctas * kc == U) {   // one whole panel per block
+    P0 = P1 = (int)blockIdx.x;
+    u_lo = (long long)P0 * kc;
+    u_hi = u_lo + kc;
+  } else if ((unsigned long long)U * (unsigned)p.ctas < (1ull << 32)) {
     const unsigned uu = (unsigned)U, nc = (unsigned)p.ctas, b = blockIdx.x;
     const unsigned lo = b * uu / nc, hi = (b + 1) * uu / nc;
     u_lo = lo;

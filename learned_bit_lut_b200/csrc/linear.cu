@@ -290,6 +290,64 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     return !(pu >= u_lo && pu + kc <= u_hi);
   };
 
+  // Row-pair modes keep the activations in L1 (evict_last) and stream the LUT
+  // and alpha/beta past it, loading alpha/beta once per group: on B200 this
+  // keeps the L1 misses, which cost several data-pipe wavefronts each, off the
+  // activation loads.
+  constexpr bool kRowPair = !C::kTr;
+
+  // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
+  // 8*blh .. 8*blh+7; every entry goes to its four bank copies
+  constexpr int kBuildPer = (512 + NCT - 1) / NCT;   // 512 tasks per panel
+  // 3- and 2-bit tables: one task per (row pair, entry), 16 << 2b tasks; the
+  // task's entry value (LUT_r[lo], LUT_r+16[hi]) is loaded a panel ahead
+  constexpr int kSmallTasks = 16 << (2 * BITS);
+  constexpr int kSmallPer = BITS == 4 ? 1 : (kSmallTasks + NCT - 1) / NCT;
+  uint32_t sv[kSmallPer], snv[kSmallPer];
+  auto load_small = [&](int P, uint32_t (&dv)[kSmallPer]) {
+#pragma unroll
+    for (int r = 0; r < kSmallPer; ++r) {
+      const int task = tid + r * NCT;
+      if (task >= kSmallTasks) break;
+      const int brp = task & 15, e = task >> 4;
+      const int br0 = (brp & 7) + 8 * (brp >> 3);
+      const int lo = e & ((1 << BITS) - 1), hi = e >> BITS;
+      const uint16_t* base_lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off) + (size_t)P * kPanelRows * 16;
+      dv[r] = ld_nc_u16(base_lut + br0 * 16 + lo) | (ld_nc_u16(base_lut + (br0 + 16) * 16 + hi) << 16);
+    }
+  };
+  const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off);
+  // this thread's LUT values of the panel being built (lw/lh) and of the
+  // next one (nw/nh), loaded a full panel ahead
+  uint4 lw[kBuildPer], nw[kBuildPer];
+  uint32_t lh[kBuildPer], nh[kBuildPer];
+  auto load_lut = [&](int P, uint4 (&dw)[kBuildPer], uint32_t (&dh)[kBuildPer]) {
+#pragma unroll
+    for (int r = 0; r < kBuildPer; ++r) {
+      const int task = tid + r * NCT;
+      if (task >= 512) break;
+      const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
+      const int br0 = (brp & 7) + 8 * (brp >> 3);
+      if (kRowPair) {
+        dw[r] = ld_stream_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
+        dh[r] = ld_stream_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+      } else {
+        dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
+        dh[r] = ld_nc_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
+      }
+    }
+  };
+  // the consumer warps' first LUT loads go out before the barrier setup
+  if (warp < NW) {
+    if (BITS == 4) {
+      load_lut(P0, lw, lh);
+      if (P0 < P1) load_lut(P0 + 1, nw, nh);
+    } else {
+      load_small(P0, sv);
+      if (P0 < P1) load_small(P0 + 1, snv);
+    }
+  }
+
   if (tid == 0) *abort = 0u;
   if (tid < NW * NS) {
     mbar_init(full_bar(tid / NS, tid % NS), 1);
@@ -400,60 +458,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 
   // =========================== consumer warps ==============================
   const int g = lane >> 2, t = lane & 3;
-  // Row-pair modes keep the activations in L1 (evict_last) and stream the LUT
-  // and alpha/beta past it, loading alpha/beta once per group: on B200 this
-  // keeps the L1 misses, which cost several data-pipe wavefronts each, off the
-  // activation loads.
-  constexpr bool kRowPair = !C::kTr;
-
-  // table build tasks: row pair brp (half, bg), high nibble bhi, low nibbles
-  // 8*blh .. 8*blh+7; every entry goes to its four bank copies
-  constexpr int kBuildPer = (512 + NCT - 1) / NCT;   // 512 tasks per panel
-  // 3- and 2-bit tables: one task per (row pair, entry), 16 << 2b tasks; the
-  // task's entry value (LUT_r[lo], LUT_r+16[hi]) is loaded a panel ahead
-  constexpr int kSmallTasks = 16 << (2 * BITS);
-  constexpr int kSmallPer = BITS == 4 ? 1 : (kSmallTasks + NCT - 1) / NCT;
-  uint32_t sv[kSmallPer], snv[kSmallPer];
-  auto load_small = [&](int P, uint32_t (&dv)[kSmallPer]) {
-#pragma unroll
-    for (int r = 0; r < kSmallPer; ++r) {
-      const int task = tid + r * NCT;
-      if (task >= kSmallTasks) break;
-      const int brp = task & 15, e = task >> 4;
-      const int br0 = (brp & 7) + 8 * (brp >> 3);
-      const int lo = e & ((1 << BITS) - 1), hi = e >> BITS;
-      const uint16_t* base_lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off) + (size_t)P * kPanelRows * 16;
-      dv[r] = ld_nc_u16(base_lut + br0 * 16 + lo) | (ld_nc_u16(base_lut + (br0 + 16) * 16 + hi) << 16);
-    }
-  };
-  const uint16_t* lut = reinterpret_cast<const uint16_t*>(p.packed + p.lut_off);
-  // this thread's LUT values of the panel being built (lw/lh) and of the
-  // next one (nw/nh), loaded a full panel ahead
-  uint4 lw[kBuildPer], nw[kBuildPer];
-  uint32_t lh[kBuildPer], nh[kBuildPer];
-  auto load_lut = [&](int P, uint4 (&dw)[kBuildPer], uint32_t (&dh)[kBuildPer]) {
-#pragma unroll
-    for (int r = 0; r < kBuildPer; ++r) {
-      const int task = tid + r * NCT;
-      if (task >= 512) break;
-      const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
-      const int br0 = (brp & 7) + 8 * (brp >> 3);
-      if (kRowPair) {
-        dw[r] = ld_stream_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
-        dh[r] = ld_stream_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
-      } else {
-        dw[r] = ld_nc_v4(lut + ((size_t)P * kPanelRows + br0) * 16 + 8 * blh);
-        dh[r] = ld_nc_u16(lut + ((size_t)P * kPanelRows + br0 + 16) * 16 + bhi);
-      }
-    }
-  };
-  if (BITS == 4) {
-    load_lut(P0, lw, lh);
-    if (P0 < P1) load_lut(P0 + 1, nw, nh);
-  } else {
-    load_small(P0, sv);
-    if (P0 < P1) load_small(P0 + 1, snv);
-  }
 
   // lookup address bases: byte b of a word goes to address bits 8..15
   const uint32_t baseA = kTabAddr | ((uint32_t)g << 4) | ((uint32_t)t << 2);   // pairs (g, g+16)

@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     const int i = w * NS + s;
     return i < n_low ? ring0 + (uint32_t)i * kSlotBytes : kHighAddr + (uint32_t)(i - n_low) * kSlotBytes;
   };
-  float* tiles = reinterpret_cast<float*>(smem + (tiles_addr - base));   // [2][NW][32][NF]
+  float* tiles = reinterpret_cast<float*>(smem + (tiles_addr - base));   // [2][NW][NF / 4][32] float4
 
   const long long U = p.units;
   const int kc = p.kc;
@@ -425,18 +425,28 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
         }
       }
       named_sync(2 + b, NCT + 32);   // tiles of panel P stored
-      const float* tb = tiles + (size_t)b * NW * 32 * NF + (size_t)lane * NF;
+      // tiles are [buffer][warp][NF / 4][lane] float4: lane-contiguous, so
+      // every 128-bit load below is free of bank conflicts
+      const float4* tb = reinterpret_cast<const float4*>(tiles) + (size_t)b * NW * (NF / 4) * 32 + lane;
       float v[NF];
 #pragma unroll
-      for (int i = 0; i < NF; ++i) {
-        float t[NW];
+      for (int i4 = 0; i4 < NF / 4; ++i4) {
+        float4 t[NW];
 #pragma unroll
-        for (int w = 0; w < NW; ++w) t[w] = tb[(size_t)w * 32 * NF + i];
+        for (int w = 0; w < NW; ++w) t[w] = tb[((size_t)w * (NF / 4) + i4) * 32];
 #pragma unroll
         for (int span = 1; span < NW; span *= 2)
 #pragma unroll
-          for (int w = 0; w + span < NW; w += 2 * span) t[w] += t[w + span];
-        v[i] = t[0];
+          for (int w = 0; w + span < NW; w += 2 * span) {
+            t[w].x += t[w + span].x;
+            t[w].y += t[w + span].y;
+            t[w].z += t[w + span].z;
+            t[w].w += t[w + span].w;
+          }
+        v[4 * i4 + 0] = t[0].x;
+        v[4 * i4 + 1] = t[0].y;
+        v[4 * i4 + 2] = t[0].z;
+        v[4 * i4 + 3] = t[0].w;
       }
       if (P + 2 <= P1) named_arrive(4 + b, NCT + 32);   // buffer b may be reused
       if (!split || finisher) {
@@ -644,10 +654,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     const int b = (P - P0) & 1;
     if (P - P0 >= 2) named_sync(4 + b, NCT + 32);   // the reducer is done with buffer b
     {
-      float4* dst = reinterpret_cast<float4*>(tiles + (size_t)b * NW * 32 * NF + (size_t)(warp * 32 + lane) * NF);
+      float4* dst = reinterpret_cast<float4*>(tiles) + ((size_t)b * NW + warp) * (NF / 4) * 32 + lane;
 #pragma unroll
-      for (int i = 0; i < NF / 4; ++i)
-        dst[i] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+      for (int i = 0; i < NF / 4; ++i) dst[(size_t)i * 32] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     }
     named_arrive(2 + b, NCT + 32);
     consumer_sync(NCT);   // every consumer is past its lookups: the tables are free

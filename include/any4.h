@@ -109,6 +109,23 @@ ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t*
 ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 
 /*
+ * any4_linear_grid - the launch geometry any4_linear / any4_linear_bits use
+ * for this shape on the current device (introspection; no launch).
+ *
+ *   bits       2, 3 or 4.
+ *   blocks     out: thread blocks of the decode kernel (M <= 16) or of the
+ *              GEMM (M > 16).
+ *   cluster    out: thread blocks per cluster. > 1 when every 32-row panel is
+ *              split along K between the blocks of one cluster, which finish
+ *              it through distributed shared memory (a shape with fewer
+ *              panels than SMs); 1 otherwise.
+ *
+ * Returns ANY4_EINVAL for null outputs, ANY4_ESHAPE for a shape or bit width
+ * the calls reject, ANY4_ECUDA if the device cannot be queried.
+ */
+ANY4_API int any4_linear_grid(int bits, int m, int n, int k, int group, int* blocks, int* cluster);
+
+/*
  * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
  *
  *   m          tokens, 1 .. 2^20. M <= 16 (decode, explainer section 3's

@@ -33,6 +33,8 @@ lib.any4_dequant.argtypes = [_p, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_dequant.restype = _c_int
 lib.any4_linear_workspace_bytes.argtypes = [_c_int, _c_int, _c_int, _c_int]
 lib.any4_linear_workspace_bytes.restype = _c_size
+lib.any4_linear_grid.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _p, _p]
+lib.any4_linear_grid.restype = _c_int
 lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
 lib.any4_linear.restype = _c_int
 lib.any4_linear_noalloc.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p]
@@ -56,7 +58,7 @@ lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
-EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
+EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes", "any4_linear_grid",
             "any4_linear", "any4_linear_noalloc", "any4_quantize", "any4_format_lut",
             "any4_pack_format", "any4_packed_bytes_bits", "any4_pack_bits", "any4_dequant_bits",
             "any4_linear_bits", "any4_strerror", "any4_last_cuda_error")
@@ -103,6 +105,13 @@ def any4_packed_bytes(n: int, k: int, group: int) -> int:
 
 def any4_linear_workspace_bytes(m: int, n: int, k: int, group: int) -> int:
     return lib.any4_linear_workspace_bytes(m, n, k, group)
+
+
+def any4_linear_grid(m: int, n: int, k: int, group: int, bits: int = 4) -> tuple[int, int]:
+    """(thread blocks, blocks per cluster) of the any4_linear launch for this shape."""
+    blocks, cluster = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib.any4_linear_grid(bits, m, n, k, group, ctypes.byref(blocks), ctypes.byref(cluster)))
+    return blocks.value, cluster.value
 
 
 def any4_pack(idx_nib: torch.Tensor, lut: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,

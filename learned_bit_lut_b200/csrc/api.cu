@@ -86,6 +86,19 @@ size_t any4_linear_workspace_bytes(int m, int n, int k, int group) {
   return any4::plan_linear(m, any4::make_layout(n, k, group), sms).workspace_bytes;
 }
 
+int any4_linear_grid(int bits, int m, int n, int k, int group, int* blocks, int* cluster) {
+  if (!blocks || !cluster) return ANY4_EINVAL;
+  if (!any4::bits_ok(bits) || m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group))
+    return ANY4_ESHAPE;
+  int sms = 0;
+  const int st = current_sm_count(&sms);
+  if (st != ANY4_OK) return st;
+  const any4::LinearPlan plan = any4::plan_linear(m, any4::make_layout(n, k, group, bits), sms);
+  *blocks = plan.ctas;
+  *cluster = plan.mode == 3 ? 1 : plan.cluster;
+  return ANY4_OK;
+}
+
 int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream) {
   if (!x || !packed || !y || !workspace) return ANY4_EINVAL;

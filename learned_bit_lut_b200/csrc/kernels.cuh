@@ -57,6 +57,7 @@ struct LinearPlan {
   int nf;               // fp32 results per lane and panel
   long long units;      // panels x K/64 chunks
   int ctas;             // persistent thread blocks (one per SM at most)
+  int cluster;          // thread blocks sharing one panel as a cluster (K slices), or 1
   size_t partials_bytes;
   size_t workspace_bytes;
 };

@@ -74,6 +74,8 @@ constexpr uint32_t kHighAddr = kTabAddr + kTabBytes;   // ring overflow and warp
 constexpr uint32_t kMaxWindowBase = 8192;    // the dynamic window starts below this
 constexpr long long kWaitLimitCycles = 4000000000ll;   // ~2 s: then the kernel records a timeout
 constexpr int kConsumerBar = 1;              // named barrier of the consumer warps
+constexpr int kMaxCluster = 8;               // thread blocks sharing one panel (portable cluster size)
+constexpr int kMinClusterChunks = 16;        // chunks a block of such a cluster works on, at least
 
 // MODE 0: M <= 4, MODE 1: M <= 8 (row-pair operands, one or two column tiles
 // of 4 tokens); MODE 2: M <= 16 (row operands, two 8-token column tiles).
@@ -91,7 +93,9 @@ struct Cfg {
   // base), the rest above them, followed by the two buffers of warp tiles
   static constexpr int kLowSlotsMin = ((int)kTabAddr - (int)kMaxWindowBase - kMiscBytes) / kSlotBytes;
   static constexpr int kHighSlotsMax = kSlots > kLowSlotsMin ? kSlots - kLowSlotsMin : 0;
-  static constexpr int kSmemBytes = (int)kHighAddr + kHighSlotsMax * kSlotBytes + 2 * kTileBytes;
+  // cluster rank 0 receives the other ranks' partial sums here
+  static constexpr int kRecvBytes = (kMaxCluster - 1) * 32 * kNF * 4;
+  static constexpr int kSmemBytes = (int)kHighAddr + kHighSlotsMax * kSlotBytes + 2 * kTileBytes + kRecvBytes;
   // everything below the tables, for a window that starts within 8 KB
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -106,6 +110,7 @@ struct Params {
   int m, n, k;
   int kc, groups, g_shift;                  // chunks per panel, groups per row, log2(G)
   int ctas;
+  int cluster;                              // thread blocks per panel (a cluster), or 1
   long long units;
   size_t w_off, lut_off, ab_off;
 };
@@ -238,16 +243,22 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   constexpr int NS = C::kNS, NF = C::kNF, NW = C::kNW, NCT = NW * 32;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
+  // In a cluster launch the shared addresses of block rank r carry r in their
+  // top byte (the block's window within the cluster's); every fixed address
+  // below (tables at 64 KB, ring overflow at 128 KB) carries the same prefix.
+  const uint32_t win = base & 0xFF000000u;
+  const uint32_t tab = win | kTabAddr;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   // Shared window: [mbarriers, flags][ring slots][row-pair tables at 64 KB]
-  // [remaining ring slots][two buffers of warp tiles]. The dynamic window
+  // [remaining ring slots][two buffers of warp tiles][cluster partials]. The dynamic window
   // starts at a small fixed offset; if it ever starts higher than planned,
   // record it and leave before touching anything else.
   const uint32_t ring0 = base + kMiscBytes;
-  const int n_low = min(C::kSlots, (int)((kTabAddr - ring0) / kSlotBytes));
-  const uint32_t tiles_addr = kHighAddr + (uint32_t)(C::kSlots - n_low) * kSlotBytes;
-  if (base > kMaxWindowBase || tiles_addr + 2u * C::kTileBytes > base + (uint32_t)C::kSmemBytes) {
+  const int n_low = min(C::kSlots, (int)((tab - ring0) / kSlotBytes));
+  const uint32_t tiles_addr = (win | kHighAddr) + (uint32_t)(C::kSlots - n_low) * kSlotBytes;
+  if (base - win > kMaxWindowBase ||
+      tiles_addr + 2u * C::kTileBytes + C::kRecvBytes > base + (uint32_t)C::kSmemBytes) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     if (tid == 0) atomicOr(p.status, 2u);
     return;
@@ -257,9 +268,16 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   auto empty_bar = [&](int w, int s) { return base + (uint32_t)(w * NS + s) * 16u + 8u; };
   auto slot_addr = [&](int w, int s) {
     const int i = w * NS + s;
-    return i < n_low ? ring0 + (uint32_t)i * kSlotBytes : kHighAddr + (uint32_t)(i - n_low) * kSlotBytes;
+    return i < n_low ? ring0 + (uint32_t)i * kSlotBytes : (win | kHighAddr) + (uint32_t)(i - n_low) * kSlotBytes;
   };
   float* tiles = reinterpret_cast<float*>(smem + (tiles_addr - base));   // [2][NW][NF / 4][32] float4
+  // A panel split across a cluster of blocks (K slices): rank 0 finishes it
+  // from the others' partials, [rank - 1][NF / 4][32] float4, which arrive as
+  // transaction bytes on its receive mbarrier.
+  const int csz = p.cluster;
+  const int crank = (int)(blockIdx.x % (unsigned)csz);
+  const uint32_t recv_addr = tiles_addr + 2u * C::kTileBytes;
+  const uint32_t recv_bar = base + 960u;
 
   const long long U = p.units;
   const int kc = p.kc;
@@ -353,8 +371,12 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     mbar_init(full_bar(tid / NS, tid % NS), 1);
     mbar_init(empty_bar(tid / NS, tid % NS), 32);
   }
+  const bool receiver = csz > 1 && crank == 0;
+  if (tid == 0 && receiver) mbar_init(recv_bar, 1);
   fence_mbar_init();
+  if (tid == 0 && receiver) mbar_arrive_expect_tx(recv_bar, (uint32_t)((csz - 1) * 32 * NF * 4));
   __syncthreads();
+  if (csz > 1) cluster_sync_all();   // rank 0's receive barrier is armed before any rank sends
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // =========================== producer warp ===============================
@@ -402,12 +424,13 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       const bool split = is_split(P);
       const long long pu = (long long)P * kc;
       const bool finisher = split && pu >= u_lo;
+      const bool clustered = csz > 1;   // split panels are finished within the cluster
       const int c_first = split ? cta_of_unit(pu, U, p.ctas) : 0;
       const int c_last = split ? cta_of_unit(pu + kc - 1, U, p.ctas) : 0;
       float other[NF];
 #pragma unroll
       for (int i = 0; i < NF; ++i) other[i] = 0.0f;
-      if (finisher && c_last > c_first) {
+      if (!clustered && finisher && c_last > c_first) {
         const unsigned need = (unsigned)(c_last - c_first);
         if (lane == 0 && ld_acquire(p.counters + P) < need) {
           const long long t0 = clock64();
@@ -450,9 +473,30 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       }
       if (P + 2 <= P1) named_arrive(4 + b, NCT + 32);   // buffer b may be reused
       if (!split || finisher) {
+        if (clustered && split) {   // the other ranks' partials, added in rank order
+          wait_bar(recv_bar, 0u, abort);
+          const float4* rb = reinterpret_cast<const float4*>(smem + (recv_addr - base)) + lane;
+          for (int r = 1; r < csz; ++r) {
+#pragma unroll
+            for (int i4 = 0; i4 < NF / 4; ++i4) {
+              const float4 q = rb[((size_t)(r - 1) * (NF / 4) + i4) * 32];
+              other[4 * i4 + 0] += q.x;
+              other[4 * i4 + 1] += q.y;
+              other[4 * i4 + 2] += q.z;
+              other[4 * i4 + 3] += q.w;
+            }
+          }
+        }
 #pragma unroll
         for (int i = 0; i < NF; ++i) store_out<MODE>(p, P, lane * NF + i, v[i] + other[i]);
-        if (split && lane == 0) p.counters[P] = 0u;   // ready for the next call
+        if (split && !clustered && lane == 0) p.counters[P] = 0u;   // ready for the next call
+      } else if (clustered) {   // send this block's partial to rank 0
+        const uint32_t bar0 = cluster_map(recv_bar, 0u);
+#pragma unroll
+        for (int i4 = 0; i4 < NF / 4; ++i4) {
+          const uint32_t dst = recv_addr + (uint32_t)((((crank - 1) * (NF / 4) + i4) * 32 + lane) * 16);
+          st_async_v4(cluster_map(dst, 0u), v[4 * i4], v[4 * i4 + 1], v[4 * i4 + 2], v[4 * i4 + 3], bar0);
+        }
       } else {
         float* dst = p.partials + ((size_t)blockIdx.x * 32 + lane) * NF;
 #pragma unroll
@@ -470,7 +514,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   const int g = lane >> 2, t = lane & 3;
 
   // lookup address bases: byte b of a word goes to address bits 8..15
-  const uint32_t baseA = kTabAddr | ((uint32_t)g << 4) | ((uint32_t)t << 2);   // pairs (g, g+16)
+  const uint32_t baseA = tab | ((uint32_t)g << 4) | ((uint32_t)t << 2);   // pairs (g, g+16)
   const uint32_t baseB = baseA | 128u;                                         // pairs (g+8, g+24)
 
   // Activation operands. Tile h serves tokens 4h.. (row-pair mode: lane g
@@ -576,7 +620,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
         const int task = tid + r * NCT;
         if (task >= kSmallTasks) break;
         const int brp = task & 15, e = task >> 4;
-        const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
+        const uint32_t bdst = tab + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
         sts128(bdst + ((uint32_t)e << 8), sv[r], sv[r], sv[r], sv[r]);
       }
 #pragma unroll
@@ -588,7 +632,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       const int task = tid + r * NCT;
       if (BITS != 4 || task >= 512) break;
       const int brp = task & 15, bhi = (task >> 4) & 15, blh = task >> 8;
-      const uint32_t bdst = kTabAddr + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
+      const uint32_t bdst = tab + ((uint32_t)(brp >> 3) << 7) + ((uint32_t)(brp & 7) << 4);
       const uint32_t L[4] = {lw[r].x, lw[r].y, lw[r].z, lw[r].w};
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -701,12 +745,66 @@ cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t st
   cfg.blockDim = dim3(Cfg<MODE>::kThreads);
   cfg.dynamicSmemBytes = Cfg<MODE>::kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)plan.cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = plan.cluster > 1 ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS>, p);
+}
+
+// How many clusters of `s` blocks of linear_kernel<MODE, BITS> the current
+// device holds at once (0 if the query fails).
+template <int MODE, int BITS>
+int active_clusters(int s) {
+  if (allow_large_smem() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)s);
+  cfg.blockDim = dim3(Cfg<MODE>::kThreads);
+  cfg.dynamicSmemBytes = Cfg<MODE>::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)s;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS>, p);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, linear_kernel<MODE, BITS>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+template <int BITS>
+int active_clusters_mode(int mode, int s) {
+  return mode == 0 ? active_clusters<0, BITS>(s) : mode == 1 ? active_clusters<1, BITS>(s) : active_clusters<2, BITS>(s);
+}
+
+// Cached per device, mode, bit width and cluster size.
+int max_active_clusters(int mode, int bits, int s) {
+  static std::atomic<int>* const cache = [] {
+    auto* c = new std::atomic<int>[64 * 3 * 3 * 4];
+    for (int i = 0; i < 64 * 3 * 3 * 4; ++i) c[i].store(-1);
+    return c;
+  }();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  const int bi = bits == 4 ? 0 : bits == 3 ? 1 : 2;
+  const int si = s == 2 ? 0 : s == 4 ? 1 : s == 8 ? 2 : 3;
+  std::atomic<int>& slot = cache[((dev * 3 + mode) * 3 + bi) * 4 + si];
+  int v = slot.load(std::memory_order_relaxed);
+  if (v < 0) {
+    v = bits == 4 ? active_clusters_mode<4>(mode, s) : bits == 3 ? active_clusters_mode<3>(mode, s)
+                                                     : active_clusters_mode<2>(mode, s);
+    slot.store(v, std::memory_order_relaxed);
+  }
+  return v;
 }
 
 template <int BITS>
@@ -732,18 +830,34 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   pl.nf = pl.mode == 0 ? 4 : pl.mode == 1 ? 8 : 16;
   pl.units = (long long)L.panels * L.kchunks;
   long long c;
+  pl.cluster = 1;
   if (L.panels <= num_sms) {
     // one whole panel per thread block: no table built for a piece of a
     // panel and no split panel to finish (on B200 this is 1.3-1.5x faster
-    // than spreading 128 panels over 148 blocks)
+    // than spreading 128 panels over 148 blocks) ...
     c = L.panels;
+    // ... and where that leaves SMs idle, a cluster of s blocks per panel,
+    // each on a K slice of at least kMinClusterChunks chunks, finishing the
+    // panel through distributed shared memory, when the device holds all
+    // the clusters at once
+    for (int s = kMaxCluster; s >= 2; s /= 2) {
+      if ((long long)L.panels * s > num_sms || L.kchunks < s * kMinClusterChunks) continue;
+      if (max_active_clusters(pl.mode, L.bits, s) < L.panels) continue;
+      pl.cluster = s;
+      c = (long long)L.panels * s;
+      break;
+    }
   } else {
     c = pl.units / kMinUnitsPerCta;
     if (c > num_sms) c = num_sms;
   }
   if (c < 1) c = 1;
   pl.ctas = (int)c;
-  pl.partials_bytes = (size_t)pl.ctas * 32 * pl.nf * sizeof(float);
+  // partial sums are only used without clusters, by at most one block per
+  // panel (whole panels) or per SM (stream-K); sized so that the workspace
+  // does not depend on the cluster decision
+  const long long pc = L.panels <= num_sms ? L.panels : c;
+  pl.partials_bytes = (size_t)(pc < 1 ? 1 : pc) * 32 * pl.nf * sizeof(float);
   pl.workspace_bytes = kHeaderBytes + pl.partials_bytes;
   return pl;
 }
@@ -767,6 +881,7 @@ cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout
   p.g_shift = 0;
   while ((1 << p.g_shift) < L.g) ++p.g_shift;
   p.ctas = plan.ctas;
+  p.cluster = plan.cluster;
   p.units = plan.units;
   p.w_off = L.w_off; p.lut_off = L.lut_off; p.ab_off = L.ab_off;
   switch (L.bits) {

@@ -126,3 +126,12 @@ def test_bits_sizes_and_rejection():
     assert a4.lib.any4_linear_bits(6, p, p, 1, 64, 64, 64, p, p, 1 << 30, None) == a4.ANY4_ESHAPE
     z = ctypes.c_void_p(0)
     assert a4.lib.any4_pack_bits(3, z, p, p, p, 64, 64, 64, p, 1 << 30, None) == a4.ANY4_EINVAL
+
+
+def test_linear_grid_rejects_on_host():
+    b, c = ctypes.c_int(0), ctypes.c_int(0)
+    assert a4.lib.any4_linear_grid(4, 1, 4096, 4096, 128, None, ctypes.byref(c)) == a4.ANY4_EINVAL
+    assert a4.lib.any4_linear_grid(4, 1, 4096, 4096, 128, ctypes.byref(b), None) == a4.ANY4_EINVAL
+    assert a4.lib.any4_linear_grid(5, 1, 4096, 4096, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_grid(4, 0, 4096, 4096, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_grid(4, 1, 4096, 4000, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE

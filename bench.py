@@ -33,11 +33,16 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 GROUP = 128
-# DRAM bytes per algorithmic byte of the linear kernel, from one ncu capture of
-# a 14336x4096, M=1, G=128 launch of the current kernel (dram__bytes_read.sum
-# 31,691,520 B, dram__bytes_write.sum 0 B, for 31,690,752 algorithmic bytes).
-# Set to None when the kernel changes.
-DRAM_PER_ALGO_BYTE = 31691520 / 31690752
+# DRAM bytes per algorithmic byte of the linear kernel from an ncu capture of
+# a 14336x4096, M=1, G=128 launch of the current kernel, or None once the
+# kernel has changed since its last capture. The kernel's warp-tile layout and
+# cluster addressing changed after the last capture (which measured
+# dram__bytes_read.sum 31,693,056 B and dram__bytes_write.sum 0 B for
+# 31,690,752 algorithmic bytes), so it is None until the next capture.
+DRAM_PER_ALGO_BYTE = None
+LAST_CAPTURE_NOTE = ("null: the kernel changed (warp-tile layout, cluster split) after its last ncu "
+                     "capture, which read 31,693,056 DRAM bytes and wrote 0 for 31,690,752 "
+                     "algorithmic bytes (14336x4096, M=1)")
 LAYERS = 32
 MS = (1, 16)
 FALLBACK_HBM_GBS = 6650.0
@@ -175,9 +180,10 @@ def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes:
                      "frac": achieved / peak,
                      "traffic": (DRAM_PER_ALGO_BYTE * step_bytes / n_calls
                                  if DRAM_PER_ALGO_BYTE is not None else None),
-                     "traffic_note": "dram bytes per launch: ncu dram__bytes_read+write of one "
-                                     "14336x4096 M=1 launch over its algorithmic bytes, times "
-                                     "this step's mean algorithmic bytes per launch",
+                     "traffic_note": ("dram bytes per launch: ncu dram__bytes_read+write of one "
+                                      "14336x4096 M=1 launch over its algorithmic bytes, times "
+                                      "this step's mean algorithmic bytes per launch"
+                                      if DRAM_PER_ALGO_BYTE is not None else LAST_CAPTURE_NOTE),
                      "peak_source": f"{peak_kind} hbm_gbs", "kernel": "linear_kernel"},
         "gpu_launches": n_calls * steps,
         "clocks": clocks,

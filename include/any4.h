@@ -148,9 +148,12 @@ ANY4_API int any4_linear_grid(int bits, int m, int n, int k, int group, int* blo
  * (fma.rn.bf16x2: the exact value rounded once to bf16) and contracted on the
  * tensor cores (mma.sync m16n8k16) with fp32 accumulation; the fp32 result
  * is rounded to bf16 nearest-even. Output rows split along K between thread
- * blocks (at most one block per SM, all resident at once) are finished by the
- * block that holds their first columns: it waits for the others' fp32
- * partials and adds them in a fixed order, so the result is deterministic.
+ * blocks (at most one block per SM, all resident at once; for shapes with
+ * few 32-row panels, the 2-8 blocks of a thread-block cluster) are finished
+ * by the block that holds their first columns: it waits for the others' fp32
+ * partials (through the workspace, or within a cluster through distributed
+ * shared memory) and adds them in a fixed order, so the result is
+ * deterministic.
  * Every wait in the kernel is bounded (~2 s); if one gives up, the kernel
  * completes without hanging and the first 32-bit word of the workspace's
  * reserved area (byte offset 65536*4) is set non-zero. It is zero after

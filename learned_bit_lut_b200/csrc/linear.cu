@@ -27,8 +27,11 @@
 //    the other row of the pair, so the MMA itself separates the rows (no data
 //    movement). For M > 8 byte permutes turn the pairs into the usual two
 //    16-row tiles, which keeps one MMA per 8 tokens.
-//  * Work split: a thread block (one per SM) owns a contiguous range of
-//    (32-row panel, 64-column chunk) units (stream-K). For each panel its
+//  * Work split: a thread block (at most one per SM) owns a contiguous range
+//    of (32-row panel, 64-column chunk) units: stream-K over all SMs when
+//    panels outnumber them, one whole panel per block when they do not, and
+//    a cluster of 2-8 blocks per panel (K slices) when whole panels would
+//    leave most SMs idle. For each panel its
 //    consumer warps (16 for M <= 4, 12 for M <= 8, 8 for M <= 16: what the
 //    register file and shared memory hold) build the 16 row-pair tables
 //    (64 KB) once, then split the panel's chunks. A producer warp streams
@@ -42,7 +45,9 @@
 //    that holds its first unit, which processes it last: it waits (bounded)
 //    for the other blocks' partials, published with a release increment when
 //    they processed the panel first, and adds them in thread-block order, so
-//    results are deterministic.
+//    results are deterministic. Within a cluster the other ranks push their
+//    partials into rank 0's shared memory (st.async onto its mbarrier)
+//    instead, and rank 0 adds them in rank order.
 //  * The SM's shared-memory/L1 data pipe (one 128-byte wavefront per clock)
 //    bounds this decode: per chunk of a panel the lookups take 32 wavefronts,
 //    the weight words about 17 (bulk-copy write plus read), the table build 8

@@ -116,36 +116,51 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
-def cpu_baseline(budget_s: float, calls=None):
-    """Time the oracle on the stack's calls, in order, for about ``budget_s``."""
-    import oracle
+def host_cores() -> int:
     try:
-        from threadpoolctl import threadpool_info
-        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        blas = 1
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float, calls=None, threads: int | None = None):
+    """Time the oracle (as it stands) on the stack's calls, in order, for about
+    ``budget_s`` seconds of work, with its BLAS limited to ``threads`` (all the
+    cores this process may run on when None). The bit-exact fp64 dequant is
+    single-threaded NumPy; the fp64 matmul uses the BLAS threads."""
+    import oracle
+    from threadpoolctl import threadpool_limits
+    cores = host_cores() if threads is None else threads
     calls = calls or stack_calls()
-    cache, xs = {}, {}
+    cache = {}
     done_bytes, t_total, count = 0, 0.0, 0
-    for (m, layer, sh) in calls:
-        key = (sh.n, sh.k)
-        if key not in cache:
-            idx, lut, a, b = synth.random_any4(sh.n, sh.k, GROUP, 0, layer=sh.name)
-            cache[key] = oracle.Any4Tensors(idx, lut, a, b, GROUP)
-        s = synth.channel_scale(sh.k, 0, layer=sh.name)
-        x = synth.activations_bf16(m, s, layer, layer=sh.name)
-        t0 = time.perf_counter()
-        oracle.linear(x, cache[key])
-        t_total += time.perf_counter() - t0
-        done_bytes += algorithmic_bytes(m, sh.n, sh.k, GROUP)
-        count += 1
-        if t_total >= budget_s:
-            break
-    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(max(1, blas)),
-            "kind": "oracle",
+    with threadpool_limits(limits=cores):
+        for (m, layer, sh) in calls:
+            key = (sh.n, sh.k)
+            if key not in cache:
+                idx, lut, a, b = synth.random_any4(sh.n, sh.k, GROUP, 0, layer=sh.name)
+                cache[key] = oracle.Any4Tensors(idx, lut, a, b, GROUP)
+            s = synth.channel_scale(sh.k, 0, layer=sh.name)
+            x = synth.activations_bf16(m, s, layer, layer=sh.name)
+            t0 = time.perf_counter()
+            oracle.linear(x, cache[key])
+            t_total += time.perf_counter() - t0
+            done_bytes += algorithmic_bytes(m, sh.n, sh.k, GROUP)
+            count += 1
+            if t_total >= budget_s:
+                break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": int(cores),
+            "kind": "oracle", "seconds": t_total, "calls": count,
             "sample": f"first {count} of {len(calls)} calls of one step (M=1 pass first), "
                       f"{t_total:.1f} s: fp64 bit-exact dequant (single-threaded numpy) + "
-                      f"fp64 matmul ({blas} BLAS threads)"}
+                      f"fp64 matmul ({cores} BLAS threads)"}
+
+
+def cpu_baselines(budget_s: float) -> dict:
+    """The oracle on all host cores, plus the same on one core."""
+    full = cpu_baseline(budget_s)
+    one = cpu_baseline(budget_s / 2, threads=1)
+    return {**full, "one_core": {k: one[k] for k in ("value", "unit", "cores", "sample")}}
 
 
 def max_over_ranks(ms: float, world: int, device) -> float:
@@ -159,6 +174,15 @@ def max_over_ranks(ms: float, world: int, device) -> float:
     return float(t.item())
 
 
+def bench_config(world: int) -> dict:
+    """The workload of the JSON line (both arms)."""
+    return {"workload": "llama3_8b_linear_stack", "layers": LAYERS,
+            "linears_per_layer": len(synth.LLAMA3_8B_LAYER), "ms": list(MS),
+            "group": GROUP, "calls_per_step": len(stack_calls()),
+            "l2": "inputs larger than L2: 3.76 GB of distinct packed weights per step",
+            "parallelism": f"replicas x{world}"}
+
+
 def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes: int, n_calls: int,
                 per_m: dict, peak: float, peak_kind: str, clocks, e2e, cpu) -> dict:
     """The JSON line of one run: whole-job throughput over all ranks (weak
@@ -169,11 +193,7 @@ def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes:
         "value": step_bytes * world / (ms_step * 1e6), "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS,
-                   "linears_per_layer": len(synth.LLAMA3_8B_LAYER), "ms": list(MS),
-                   "group": GROUP, "calls_per_step": n_calls,
-                   "l2": "inputs larger than L2: 3.76 GB of distinct packed weights per step",
-                   "parallelism": f"replicas x{world}"},
+        "config": bench_config(world),
         "us_per_call": ms_step * 1e3 / n_calls,
         "by_m": per_m,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -193,28 +213,85 @@ def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes:
 
 
 def run_reference(args, rank: int, world: int):
+    """The oracle on the host cores, rank 0 only: each step is a bounded
+    sample of the stack's calls (in order); ``value`` is the algorithmic bytes
+    of the sampled calls over the time they took, ``ms_per_step`` the measured
+    time of one sampled step."""
     if rank != 0:
         return
     calls = stack_calls()
-    step_bytes_full = sum(algorithmic_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
     per_step_budget = max(0.5, 60.0 / max(1, args.steps + args.warmup))
     vals = []
     for i in range(args.warmup + args.steps):
         r = cpu_baseline(per_step_budget, calls)
         if i >= args.warmup:
             vals.append(r)
-    value = float(np.mean([v["value"] for v in vals]))
-    ms_per_step = step_bytes_full / (value * 1e9) * 1e3
+    seconds = sum(v["seconds"] for v in vals)
+    value = sum(v["value"] * v["seconds"] for v in vals) / seconds
     line = {"impl": "reference", "metric": "any4_linear achieved HBM GB/s (algorithmic bytes)",
             "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": seconds * 1e3 / len(vals), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "llama3_8b_linear_stack", "layers": LAYERS, "ms": list(MS),
-                       "group": GROUP, "calls_per_step": len(calls)},
+            "config": bench_config(1),
+            "step": (f"a bounded sample of the stack: the first {vals[-1]['calls']} of {len(calls)} "
+                     f"calls, about {per_step_budget:.1f} s of oracle work per step"),
             "cpu_baseline": {**vals[-1], "value": value},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# Shapes of the per-shape lines: the Llama-3-8B MLP shapes the 70 % target is
+# set on, then the attention projections.
+BY_SHAPE = (("gate/up", 14336, 4096), ("down", 4096, 14336), ("q/o", 4096, 4096), ("k/v", 1024, 4096))
+L2_BYTES = 126 * 2 ** 20
+
+
+def time_by_shape(a4, dev, peak: float, calls: int = 200) -> dict:
+    """µs per call of each shape at M = 1 and 16: ``calls`` back-to-back
+    any4_linear launches replayed from one CUDA graph, rotating over enough
+    distinct copies of the packed weight (>= 3x the L2 size) that every call
+    reads its weight from HBM; CUDA events around the replay."""
+    import torch
+    out = {}
+    for name, n, k in BY_SHAPE:
+        idx, lut, al, be = synth.random_any4(n, k, GROUP, 0, layer="shape_" + name)
+        t = lambda a: torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+        base = a4.any4_pack(t(idx), t(lut), t(al), t(be), GROUP)
+        wbytes = algorithmic_bytes(1, n, k, GROUP)
+        copies = max(2, -(-3 * L2_BYTES // wbytes))
+        packs = [base] + [base.clone() for _ in range(copies - 1)]
+        for m in MS:
+            s = synth.channel_scale(k, 0, layer="shape_" + name)
+            x = torch.from_numpy(synth.activations_bf16(m, s, 7, layer="shape_" + name).view(np.int16)).to(dev).view(torch.bfloat16)
+            y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            ws = torch.zeros(a4.any4_linear_workspace_bytes(m, n, k, GROUP), dtype=torch.uint8, device=dev)
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                for i in range(4):
+                    a4.any4_linear(x, packs[i % copies], n, k, GROUP, out=y, workspace=ws)
+            torch.cuda.current_stream(dev).wait_stream(side)
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(calls):
+                    a4.any4_linear(x, packs[i % copies], n, k, GROUP, out=y, workspace=ws)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            g.replay()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            us = e0.elapsed_time(e1) * 1e3 / calls
+            b = algorithmic_bytes(m, n, k, GROUP)
+            out[f"{name} {n}x{k} M={m}"] = {"us_per_call": us, "GB/s": b / (us * 1e3),
+                                             "frac": b / (us * 1e3) / peak, "weight_copies": copies}
+            del g
+        del packs, base
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args, rank: int, world: int, local_rank: int):
@@ -308,6 +385,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     step_bytes = sum(algorithmic_bytes(m, sh.n, sh.k, GROUP) for m, _, sh in calls)
     peak, peak_kind = read_peaks()
+    by_shape = None if args.no_shapes else time_by_shape(a4, dev, peak)
 
     # end to end through the Python API: pinned host x in, y out, every step
     e2e = None
@@ -335,11 +413,12 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        cpu = cpu_baseline(args.cpu_seconds)
+        cpu = cpu_baselines(args.cpu_seconds)
 
     if rank == 0:
         line = result_line(world, args.steps, args.warmup, ms_step, step_bytes, len(calls), per_m,
                            peak, peak_kind, sampler.summary(), e2e, cpu)
+        line["by_shape"] = by_shape
         print(json.dumps(line), flush=True)
     for g in graphs.values():
         del g
@@ -371,12 +450,21 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-shapes", action="store_true", help="skip the per-shape lines")
+    ap.add_argument("--shapes", action="store_true", help="only the per-shape lines (1 GPU)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--one", type=int, nargs=4, metavar=("N", "K", "M", "G"),
                     help="only run a few calls of one shape (profiler captures)")
     args = ap.parse_args()
     if args.one:
         run_one(*args.one)
+        return
+    if args.shapes:
+        import torch
+
+        import learned_bit_lut_b200 as a4
+        peak, _ = read_peaks()
+        print(json.dumps(time_by_shape(a4, torch.device("cuda:0"), peak)), flush=True)
         return
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -192,20 +192,37 @@ ANY4_API int any4_linear_bits(int bits, const uint16_t* x, const void* packed, i
  * latency-critical loops that must not call cudaMalloc because it can
  * synchronize the device.
  *
- * Same arguments, result and rounding as any4_linear, minus the workspace:
- * the partial sums and counters live in a fixed 8 MiB array of device memory
+ * Same arguments, result and rounding as any4_linear for 1 <= M <= 16, minus
+ * the workspace (M > 16, the prefill path, returns ANY4_ESHAPE): the partial
+ * sums, counters and status word live in a fixed 8 MiB array of device memory
  * that this library reserves on every GPU that loads it, until the process
- * exits. A shape whose launch needs more than that returns ANY4_EWORKSPACE
- * (on a 148-SM B200 all accepted shapes fit). The call allocates and frees
- * nothing. The first call on a device looks up the array's address with that
- * device current, so make it before any stream capture on that device. All
- * calls on a device share the array: each call clears the counters it uses
- * on `stream` before its kernel, and calls that can run at the same time on
- * the GPU race and must be ordered by the caller. On ANY4_ECUDA the CUDA
- * error code is not recorded for any4_last_cuda_error().
+ * exits. A shape whose launch needs more than that returns ANY4_EWORKSPACE;
+ * the largest need is 256 KiB + 256 B plus 2,048 bytes per SM (M = 9..16),
+ * 0.56 MB on a 148-SM B200, so every accepted shape fits. The call allocates
+ * and frees nothing. The first call on a
+ * device (of this function or any4_noalloc_status_word) looks up the array's
+ * address with that device current, so make it before any stream capture on
+ * that device. All calls on a device share the array: each call first clears
+ * its header (counters and status word) on `stream`, and calls that can run
+ * at the same time on the GPU race and must be ordered by the caller.
+ * A bounded wait inside the kernel that gave up leaves y incomplete and sets
+ * the status word non-zero; the call itself still returns ANY4_OK (it only
+ * enqueues work). Read the word through any4_noalloc_status_word() after the
+ * call's work on `stream` has completed.
  */
 ANY4_API int any4_linear_noalloc(const uint16_t* x, const void* packed, int m, int n, int k,
                                  int group, uint16_t* y, any4_stream_t stream);
+
+/*
+ * any4_noalloc_status_word - device address (on the current device) of the
+ * 32-bit status word of any4_linear_noalloc: 0 after a call that completed
+ * normally, non-zero (bit 0: a bounded wait timed out) otherwise, until the
+ * next any4_linear_noalloc call on that device clears it. Host-only lookup;
+ * copy the word with any device-to-host copy of the caller's choice.
+ * Returns ANY4_OK, ANY4_EINVAL for a NULL status, ANY4_ECUDA if the device
+ * cannot be queried.
+ */
+ANY4_API int any4_noalloc_status_word(const uint32_t** status);
 
 /*
  * any4_quantize - the any4 quantizer on the GPU (explainer sections 2.1 and

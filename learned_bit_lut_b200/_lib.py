@@ -39,6 +39,8 @@ lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_s
 lib.any4_linear.restype = _c_int
 lib.any4_linear_noalloc.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_linear_noalloc.restype = _c_int
+lib.any4_noalloc_status_word.argtypes = [ctypes.POINTER(_p)]
+lib.any4_noalloc_status_word.restype = _c_int
 lib.any4_format_lut.argtypes = [_c_int, _p]
 lib.any4_format_lut.restype = _c_int
 lib.any4_pack_format.argtypes = [_c_int, _p, _p, _p, _c_int, _c_int, _c_int, _p, _c_size, _p]
@@ -59,7 +61,7 @@ lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes", "any4_linear_grid",
-            "any4_linear", "any4_linear_noalloc", "any4_quantize", "any4_format_lut",
+            "any4_linear", "any4_linear_noalloc", "any4_noalloc_status_word", "any4_quantize", "any4_format_lut",
             "any4_pack_format", "any4_packed_bytes_bits", "any4_pack_bits", "any4_dequant_bits",
             "any4_linear_bits", "any4_strerror", "any4_last_cuda_error")
 
@@ -234,6 +236,26 @@ def any4_linear_noalloc(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, g
     _check(lib.any4_linear_noalloc(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k,
                                    group, _dev(out, "out", 2, (m, n)), _stream(x.device)))
     return out
+
+
+class _DeviceWord:
+    """A 32-bit device word exposed through the CUDA array interface."""
+
+    def __init__(self, ptr: int):
+        self.__cuda_array_interface__ = {"shape": (1,), "typestr": "<u4", "data": (ptr, False),
+                                         "version": 3}
+
+
+def noalloc_status(device: torch.device | None = None) -> int:
+    """The status word of any4_linear_noalloc on ``device`` (0: the last call
+    completed normally). Synchronizes that device before reading it."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        ptr = _p()
+        _check(lib.any4_noalloc_status_word(ctypes.byref(ptr)))
+        torch.cuda.synchronize(dev)
+        word = torch.as_tensor(_DeviceWord(ptr.value), device=dev)
+        return int(word.view(torch.int32).item()) & 0xFFFFFFFF
 
 
 def any4_quantize(w: torch.Tensor, ex: torch.Tensor, group: int, bits: int = 4,

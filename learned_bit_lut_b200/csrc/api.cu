@@ -23,30 +23,43 @@ int fail_cuda(cudaError_t e) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// SM count of the current device, or a negative status.
+}  // namespace
+
+namespace any4 {
+cudaError_t cached_sm_count(int* sms);
+}
+
+namespace {
+
+// SM count of the current device (cached per device), or a negative status.
 int current_sm_count(int* sms) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail_cuda(e);
-  if (dev >= 0 && dev < kMaxDevices) {
-    const int c = g_sm_count[dev].load(std::memory_order_relaxed);
-    if (c > 0) {
-      *sms = c;
-      return ANY4_OK;
-    }
-  }
-  int c = 0;
-  e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return fail_cuda(e);
-  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(c, std::memory_order_relaxed);
-  *sms = c;
-  return ANY4_OK;
+  const cudaError_t e = any4::cached_sm_count(sms);
+  return e == cudaSuccess ? ANY4_OK : fail_cuda(e);
 }
 
 }  // namespace
 
 namespace any4 {
 int record_cuda_error(cudaError_t e) { return fail_cuda(e); }
+
+cudaError_t cached_sm_count(int* sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int c = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (c > 0) {
+      *sms = c;
+      return cudaSuccess;
+    }
+  }
+  int c = 0;
+  e = cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(c, std::memory_order_relaxed);
+  *sms = c;
+  return cudaSuccess;
+}
 }  // namespace any4
 
 extern "C" {

@@ -27,6 +27,9 @@ cudaError_t launch_quantize(const uint16_t* w, const double* ex, int n, int k, i
 // Keeps e for any4_last_cuda_error() on this host thread; returns ANY4_ECUDA.
 int record_cuda_error(cudaError_t e);
 
+// SM count of the current device, queried once per device and cached.
+cudaError_t cached_sm_count(int* sms);
+
 // The 16 bf16 values of a fixed-table format (any4_format); false if unknown.
 bool format_table(int format, uint16_t (&lut)[16]);
 

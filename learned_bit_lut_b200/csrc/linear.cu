@@ -197,6 +197,22 @@ __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
+// End of a clustered launch, reached by every warp of every block: no block
+// leaves while another block of its cluster may still store into its shared
+// memory. The cluster barrier orders the other ranks' st.async issue before
+// rank 0's exit; a rank 0 that gave up waiting for their partials (a timeout)
+// then waits once more, bounded, for the bytes to land.
+__device__ __forceinline__ void cluster_tail(int csz, bool receiver, uint32_t recv_bar) {
+  if (csz <= 1) return;
+  __syncwarp();
+  cluster_sync_all();
+  if (receiver && !mbar_try_wait(recv_bar, 0u)) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(recv_bar, 0u) && clock64() - t0 < kWaitLimitCycles) {
+    }
+  }
+}
+
 // (token, row within the panel) of result i of lane `ln`.
 template <int MODE>
 __device__ __forceinline__ void out_pos(int ln, int i, int& token, int& row) {
@@ -410,6 +426,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       cur.c += n;
       cur.settle();
     }
+    cluster_tail(csz, receiver, recv_bar);
     return;
   }
 
@@ -512,6 +529,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       }
     }
     if (lane == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
+    cluster_tail(csz, receiver, recv_bar);
     return;
   }
 
@@ -711,6 +729,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     consumer_sync(NCT);   // every consumer is past its lookups: the tables are free
   }
   if (tid == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
+  cluster_tail(csz, receiver, recv_bar);
 }
 
 template <int MODE, int BITS>

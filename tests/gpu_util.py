@@ -66,11 +66,20 @@ def mixed(n: int, k: int, g: int, rows: tuple, seed: int = 0, layer: str = "w",
     return oracle.Any4Tensors(idx, lut, a, b, g), s
 
 
-def sample_rows(n: int, count: int = 48, seed: int = 0) -> tuple:
-    """Rows of the first and last tiles plus spread random rows."""
+def sample_rows(n: int, count: int = 48, seed: int = 0, whole_panels: int = 4) -> tuple:
+    """Rows of the first and last tiles, spread random rows, and every row of
+    ``whole_panels`` 32-row panels (the first, the last and random ones).
+
+    At the benchmark shapes every panel of the any4 decode kernel is split
+    along K between several warps and finished by the last one to arrive, so
+    whole panels check that reduction element by element."""
     g = np.random.default_rng(seed)
     pick = set(range(min(16, n))) | set(range(max(0, n - 16), n))
     pick |= set(g.choice(n, size=min(n, count), replace=False).tolist())
+    panels = (n + 31) // 32
+    chosen = {0, panels - 1} | set(g.choice(panels, size=min(panels, max(0, whole_panels - 2)), replace=False).tolist())
+    for p in sorted(chosen):
+        pick |= set(range(32 * p, min(n, 32 * p + 32)))
     return tuple(sorted(pick))
 
 

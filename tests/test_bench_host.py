@@ -88,3 +88,9 @@ def test_reference_arm_other_ranks_do_no_work(capsys):
         steps, warmup, gpus = 1, 0, 2
     assert bench.run_reference(A(), rank=1, world=2) is None
     assert capsys.readouterr().out == ""
+
+
+def test_both_arms_share_the_config():
+    one = bench.result_line(1, 200, 5, 5.0, 7_592_738_816, 448, {}, 6457.4, "measured", {}, None, None)
+    assert one["config"] == bench.bench_config(1)
+    assert one["config"]["calls_per_step"] == 448

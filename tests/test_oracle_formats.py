@@ -25,6 +25,16 @@ def test_int4_table_is_the_grid():
     np.testing.assert_array_equal(ob.bf16_bits_to_f64(bits), np.arange(-8.0, 8.0))
 
 
+def test_nf4_levels_equal_published_values():
+    # tests/golden/nf4_levels.json: the NF4 values as published with QLoRA
+    import json
+    import os
+    gold = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "nf4_levels.json")))
+    pub = np.array(gold["values"], dtype=np.float64)
+    np.testing.assert_allclose(oracle.nf4_levels(), pub, rtol=0, atol=gold["abs_tolerance_float64"])
+    np.testing.assert_array_equal(oracle.format_lut_bits("nf4"), oracle.f64_to_bf16_bits(pub))
+
+
 def test_nf4_table_properties():
     v = ob.bf16_bits_to_f64(oracle.format_lut_bits("nf4"))
     assert np.all(np.diff(v) > 0) and v[0] == -1.0 and v[-1] == 1.0

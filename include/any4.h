@@ -103,8 +103,9 @@ ANY4_API int any4_dequant(const void* packed, int n, int k, int group, uint16_t*
  * accepted. The workspace holds a fixed header of 65536 arrival counters (one
  * per possible 16-row tile) and a reserved 256-byte area, then the fp32
  * partial sums of output blocks split along K between thread blocks. For
- * M > 16 (prefill) the header is followed by a bf16 N x K scratch for the
- * dequantized weight instead (N*K*2 bytes, rounded up to 256).
+ * M > 512 (prefill beyond the fused decode) the header is followed by a bf16
+ * N x K scratch for the dequantized weight (N*K*2 bytes, rounded up to 256),
+ * then the partial sums.
  */
 ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
 
@@ -129,10 +130,13 @@ ANY4_API int any4_linear_grid(int bits, int m, int n, int k, int group, int* blo
  * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
  *
  *   m          tokens, 1 .. 2^20. M <= 16 (decode, explainer section 3's
- *              batch 1-16) runs the fused dequant-and-contract kernel below;
- *              M > 16 (prefill) dequantizes W once into the workspace (the
- *              bit-exact any4_dequant values) and runs a tensor-core GEMM
- *              (tcgen05, fp32 accumulation in tensor memory).
+ *              batch 1-16) runs the fused dequant-and-contract kernel below.
+ *              M > 16 (prefill) runs a tensor-core GEMM (tcgen05, fp32
+ *              accumulation in tensor memory): up to M = 512 its A tiles are
+ *              decoded from the packed weight straight into shared memory
+ *              (w_hat rounded once to bf16, as below); beyond that W is
+ *              dequantized once into the workspace (the bit-exact
+ *              any4_dequant values) and the GEMM reads it back.
  *   x          [M][K] bf16 activations, row-major, 16-byte aligned.
  *   packed     the any4_pack output for W (N x K, group G).
  *   y          [M][N] bf16 output, row-major, 4-byte aligned.
@@ -171,9 +175,13 @@ ANY4_API int any4_linear(const uint16_t* x, const void* packed, int m, int n, in
  * with bits = 3 or 2 produces them. The packed buffer stores each row pair's
  * two indices as one 2b-bit code, densely (N*K*b/8 bytes of indices) and is
  * only valid for the *_bits calls with the same b. bits = 4 is the same as
- * the plain calls. Workspace sizes are those of any4_linear_workspace_bytes.
- * Errors as for the plain calls, plus ANY4_ESHAPE for bits not in {2, 3, 4}.
+ * the plain calls. any4_linear_bits needs any4_linear_workspace_bytes_bits
+ * bytes of workspace: for M > 16, b = 3 and 2 dequantize W into the
+ * workspace (N*K*2 bytes more than any4, whose prefill decodes on the fly up
+ * to 512 tokens). Errors as for the plain calls, plus ANY4_ESHAPE for bits
+ * not in {2, 3, 4}; the size query returns 0 for those.
  */
+ANY4_API size_t any4_linear_workspace_bytes_bits(int bits, int m, int n, int k, int group);
 ANY4_API size_t any4_packed_bytes_bits(int bits, int n, int k, int group);
 ANY4_API int any4_pack_bits(int bits, const uint8_t* idx_nib, const uint16_t* lut,
                             const uint16_t* alpha, const uint16_t* beta, int n, int k, int group,

@@ -33,6 +33,8 @@ lib.any4_dequant.argtypes = [_p, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_dequant.restype = _c_int
 lib.any4_linear_workspace_bytes.argtypes = [_c_int, _c_int, _c_int, _c_int]
 lib.any4_linear_workspace_bytes.restype = _c_size
+lib.any4_linear_workspace_bytes_bits.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int]
+lib.any4_linear_workspace_bytes_bits.restype = _c_size
 lib.any4_linear_grid.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_linear_grid.restype = _c_int
 lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
@@ -60,7 +62,8 @@ lib.any4_strerror.restype = ctypes.c_char_p
 lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
-EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes", "any4_linear_grid",
+EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
+            "any4_linear_workspace_bytes_bits", "any4_linear_grid",
             "any4_linear", "any4_linear_noalloc", "any4_noalloc_status_word", "any4_quantize", "any4_format_lut",
             "any4_pack_format", "any4_packed_bytes_bits", "any4_pack_bits", "any4_dequant_bits",
             "any4_linear_bits", "any4_strerror", "any4_last_cuda_error")
@@ -172,7 +175,7 @@ def any4_linear_bits(bits: int, x: torch.Tensor, packed: torch.Tensor, n: int, k
     if out is None:
         out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
-        workspace = workspace_for(m, n, k, group, x.device)
+        workspace = workspace_for(m, n, k, group, x.device, bits)
     _check(lib.any4_linear_bits(bits, _dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
                                 _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
                                 workspace.numel(), _stream(x.device)))
@@ -192,10 +195,10 @@ def any4_dequant(packed: torch.Tensor, n: int, k: int, group: int,
 _WORKSPACES: dict = {}
 
 
-def workspace_for(m: int, n: int, k: int, group: int, device: torch.device) -> torch.Tensor:
+def workspace_for(m: int, n: int, k: int, group: int, device: torch.device, bits: int = 4) -> torch.Tensor:
     """A zero-initialised workspace for this stream, grown on demand and reused
     by later calls on the same stream (calls on one stream never overlap)."""
-    need = any4_linear_workspace_bytes(m, n, k, group)
+    need = lib.any4_linear_workspace_bytes_bits(bits, m, n, k, group)
     if need == 0:
         raise Any4Error(ANY4_ESHAPE)
     key = (device.index if device.index is not None else torch.cuda.current_device(),

@@ -99,6 +99,13 @@ size_t any4_linear_workspace_bytes(int m, int n, int k, int group) {
   return any4::plan_linear(m, any4::make_layout(n, k, group), sms).workspace_bytes;
 }
 
+size_t any4_linear_workspace_bytes_bits(int bits, int m, int n, int k, int group) {
+  if (!any4::bits_ok(bits) || m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group)) return 0;
+  int sms = 0;
+  if (current_sm_count(&sms) != ANY4_OK) return 0;
+  return any4::plan_linear(m, any4::make_layout(n, k, group, bits), sms).workspace_bytes;
+}
+
 int any4_linear_grid(int bits, int m, int n, int k, int group, int* blocks, int* cluster) {
   if (!blocks || !cluster) return ANY4_EINVAL;
   if (!any4::bits_ok(bits) || m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group))

@@ -197,18 +197,19 @@ __device__ __forceinline__ void wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// End of a clustered launch, reached by every warp of every block: no block
-// leaves while another block of its cluster may still store into its shared
-// memory. The cluster barrier orders the other ranks' st.async issue before
-// rank 0's exit; a rank 0 that gave up waiting for their partials (a timeout)
-// then waits once more, bounded, for the bytes to land.
-__device__ __forceinline__ void cluster_tail(int csz, bool receiver, uint32_t recv_bar) {
-  if (csz <= 1) return;
-  __syncwarp();
-  cluster_sync_all();
-  if (receiver && !mbar_try_wait(recv_bar, 0u)) {
-    const long long t0 = clock64();
-    while (!mbar_try_wait(recv_bar, 0u) && clock64() - t0 < kWaitLimitCycles) {
+// Rank 0 of a cluster waits for the other ranks' partials: every rank sends
+// its partial even after a timeout of its own (then with whatever it summed),
+// so this wait ends once their bytes have landed. It is bounded (twice the
+// other waits, so a rank that gives up one of its own waits still gets to
+// send) but, unlike wait_bar, not cut short by this block's abort flag: rank 0
+// must not exit while another rank may still store into its shared memory.
+__device__ __forceinline__ void wait_partials(uint32_t bar, volatile uint32_t* abort) {
+  if (mbar_try_wait(bar, 0u)) return;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, 0u)) {
+    if (clock64() - t0 > 2 * kWaitLimitCycles) {
+      *abort = 1u;
+      return;
     }
   }
 }
@@ -426,7 +427,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       cur.c += n;
       cur.settle();
     }
-    cluster_tail(csz, receiver, recv_bar);
     return;
   }
 
@@ -496,7 +496,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       if (P + 2 <= P1) named_arrive(4 + b, NCT + 32);   // buffer b may be reused
       if (!split || finisher) {
         if (clustered && split) {   // the other ranks' partials, added in rank order
-          wait_bar(recv_bar, 0u, abort);
+          wait_partials(recv_bar, abort);
           const float4* rb = reinterpret_cast<const float4*>(smem + (recv_addr - base)) + lane;
           for (int r = 1; r < csz; ++r) {
 #pragma unroll
@@ -529,7 +529,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
       }
     }
     if (lane == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
-    cluster_tail(csz, receiver, recv_bar);
     return;
   }
 
@@ -729,7 +728,6 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     consumer_sync(NCT);   // every consumer is past its lookups: the tables are free
   }
   if (tid == 0 && *abort) atomicOr(p.status, kStatusWaitTimeout);
-  cluster_tail(csz, receiver, recv_bar);
 }
 
 template <int MODE, int BITS>

@@ -1,9 +1,15 @@
-"""GPU parity of the prefill path (M > 16): the bf16 W_hat scratch must equal
-any4_dequant bit for bit, and y must meet the linear layer's acceptance bar
-and the tight elementwise bar (the GEMM contracts the same bf16 weights with
-fp32 accumulation). Shapes cover one tile, ragged token and row tails, K not
-a multiple of the 64-column stage count of a tile, every group size, and the
-Llama-3-8B MLP shapes at full size (sampled rows)."""
+"""GPU parity of the prefill path (M > 16).
+
+any4 up to 512 tokens decodes each 128-row weight tile straight into the
+tensor-core GEMM's shared-memory stages (row tables in registers, no bf16
+copy of W); any4 beyond 512 tokens and any3 / any2 dequantize into a
+workspace scratch first, which must equal any4_dequant_bits bit for bit. y must meet the linear layer's acceptance bar
+and the tight elementwise bar (both paths contract bf16 weights with fp32
+accumulation). Shapes cover every token-tile width of the fused path (64,
+128, 256 and several 256-token tiles), ragged token and row tails (a last
+128-row tile with panels past N), K not a multiple of a tile's stage count,
+every group size, split-K, and the Llama-3-8B MLP shapes at full size
+(sampled rows, whole panels among them)."""
 import numpy as np
 import pytest
 import torch
@@ -24,8 +30,10 @@ def _gpu():
 
 
 @pytest.mark.parametrize("n,k,g,m", [(256, 512, 128, 17), (256, 512, 128, 64), (16, 64, 64, 17),
+                                     (256, 512, 128, 65), (256, 512, 128, 128), (256, 512, 128, 129),
                                      (1024, 4096, 128, 256), (160, 2112, 64, 300),
-                                     (4096, 1024, 256, 33), (48, 1024, 1024, 513), (272, 1536, 512, 257)])
+                                     (4096, 1024, 256, 33), (48, 1024, 1024, 513), (272, 1536, 512, 257),
+                                     (2080, 1024, 128, 96), (256, 1024, 128, 512)])
 def test_prefill_shapes(n, k, g, m):
     q, s = quantized(n, k, g, layer=f"pre{n}x{k}", iters=4)
     x = synth.activations_bf16(m, s, 7, layer=f"pre{n}x{k}")
@@ -46,18 +54,24 @@ def test_prefill_llama3_8b_mlp_sampled(shape, m):
     check_linear(y, x, q, rows)
 
 
-def test_prefill_scratch_is_the_dequantized_weight():
+def test_prefill_scratch_is_the_dequantized_weight_any3():
+    from gpu_util import calib, to_dev
+    import oracle
     n, k, g, m = 1024, 2048, 128, 40
-    q, s = quantized(n, k, g, layer="pscratch", iters=4)
-    x = synth.activations_bf16(m, s, 9, layer="pscratch")
-    packed = pack_dev(q)
-    ws = a4.workspace_for(m, n, k, g, torch.device("cuda:0"))
-    a4.any4_linear(bf16_dev(x), packed, n, k, g, workspace=ws)
-    w = a4.any4_dequant(packed, n, k, g)
+    w = synth.weights_bf16(n, k, 0, layer="pscratch3")
+    s, ex = calib(k, 0, "pscratch3")
+    q = oracle.quantize(w, ex, g, iters=4, bits=3)
+    x = synth.activations_bf16(m, s, 9, layer="pscratch3")
+    packed = a4.any4_pack_bits(3, to_dev(q.idx_nib), to_dev(q.lut), to_dev(q.alpha), to_dev(q.beta), g)
+    ws = a4.workspace_for(m, n, k, g, torch.device("cuda:0"), bits=3)
+    assert a4.lib.any4_linear_workspace_bytes_bits(3, m, n, k, g) >= STATUS_OFFSET + 256 + n * k * 2
+    y = a4.any4_linear_bits(3, bf16_dev(x), packed, n, k, g, workspace=ws)
+    wd = a4.any4_dequant_bits(3, packed, n, k, g)
     torch.cuda.synchronize()
     off = STATUS_OFFSET + 256
     scratch = ws[off:off + n * k * 2].view(torch.int16).view(n, k)
-    assert torch.equal(scratch, w.view(torch.int16))
+    assert torch.equal(scratch, wd.view(torch.int16))
+    check_linear(y, x, q)
 
 
 def test_prefill_repeatable_and_guard_rows_untouched():
@@ -77,8 +91,10 @@ def test_prefill_repeatable_and_guard_rows_untouched():
 
 def test_prefill_workspace_size():
     n, k, g = 4096, 4096, 128
+    header = STATUS_OFFSET + 256
     need = a4.any4_linear_workspace_bytes(17, n, k, g)
-    assert need >= STATUS_OFFSET + 256 + n * k * 2
+    assert header <= need < header + n * k * 2          # any4: no dequantized copy of W
+    assert a4.lib.any4_linear_workspace_bytes(17, n, k, g) == need
     x = torch.zeros((17, k), dtype=torch.bfloat16, device="cuda:0")
     y = torch.empty((17, n), dtype=torch.bfloat16, device="cuda:0")
     packed = torch.zeros(a4.any4_packed_bytes(n, k, g), dtype=torch.uint8, device="cuda:0")

@@ -61,11 +61,19 @@ struct LinearPlan {
   long long units;      // panels x K/64 chunks
   int ctas;             // persistent thread blocks (one per SM at most)
   int cluster;          // thread blocks sharing one panel as a cluster (K slices), or 1
+  bool regt;            // register-table kernel (linear_regt.cu) instead of linear.cu's
   size_t partials_bytes;
   size_t workspace_bytes;
 };
 
 LinearPlan plan_linear(int m, const Layout& L, int num_sms);
+
+// M <= 16, any4, few chunks per thread block: row tables in registers, one
+// cluster of `cluster` blocks per panel (linear_regt.cu).
+int regt_warps(int m);
+int regt_max_cluster();
+cudaError_t launch_linear_regt(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
+                               void* workspace, int cluster, cudaStream_t stream);
 
 cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout& L, int m,
                           uint16_t* y, void* workspace, const LinearPlan& plan,

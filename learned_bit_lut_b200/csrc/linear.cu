@@ -81,6 +81,7 @@ constexpr long long kWaitLimitCycles = 4000000000ll;   // ~2 s: then the kernel 
 constexpr int kConsumerBar = 1;              // named barrier of the consumer warps
 constexpr int kMaxCluster = 8;               // thread blocks sharing one panel (portable cluster size)
 constexpr int kMinClusterChunks = 16;        // chunks a block of such a cluster works on, at least
+constexpr int kRegtMaxChunks = 16;           // chunks per block up to which linear_regt.cu decodes
 
 // MODE 0: M <= 4, MODE 1: M <= 8 (row-pair operands, one or two column tiles
 // of 4 tokens); MODE 2: M <= 16 (row operands, two 8-token column tiles).
@@ -875,6 +876,25 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   }
   if (c < 1) c = 1;
   pl.ctas = (int)c;
+  // a short K split over a cluster per panel (at most kRegtMaxChunks chunks
+  // per block, at least one per warp): the fixed cost of a panel's shared
+  // tables and barriers outweighs the decode, so the register-table kernel
+  // takes it, on its own cluster split (measured on B200: faster on such
+  // shapes, slower without a cluster or with idle warps)
+  if (L.bits == 4 && L.panels <= num_sms) {
+    int s = 0;
+    for (int q = regt_max_cluster(); q >= 2; q /= 2) {
+      if ((long long)L.panels * q <= num_sms && L.kchunks >= q * regt_warps(m)) {
+        s = q;
+        break;
+      }
+    }
+    if (s > 0 && L.kchunks <= s * kRegtMaxChunks) {
+      pl.regt = true;
+      pl.cluster = s;
+      pl.ctas = L.panels * s;
+    }
+  }
   // partial sums are only used without clusters, by at most one block per
   // panel (whole panels) or per SM (stream-K); sized so that the workspace
   // does not depend on the cluster decision
@@ -888,6 +908,7 @@ cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout
                           uint16_t* y, void* workspace, const LinearPlan& plan,
                           cudaStream_t stream) {
   if (plan.mode == 3) return launch_prefill(x, packed, L, m, y, workspace, plan.ctas, stream);
+  if (plan.regt) return launch_linear_regt(x, packed, L, m, y, workspace, plan.cluster, stream);
   cudaError_t e = allow_large_smem();
   if (e != cudaSuccess) return e;
   Params p{};

@@ -4,7 +4,11 @@ on a K slice, and the cluster's first block adds the others' fp32 partials
 (received through distributed shared memory) in rank order. Checks that the
 launch really is clustered, the linear layer's acceptance bar against the
 oracle for every decode mode (M = 1, 3, 8, 16), ragged K slices and a ragged
-last panel, any3 / any2, and that repeated calls are bit-identical."""
+last panel, any3 / any2, and that repeated calls are bit-identical. For any4
+the shapes with at most 16 chunks per block (1024 x 4096, 1008 x 4096 and
+2048 x 2048) take the register-table kernel, which splits the same
+way (tests/test_gpu_regt.py); the others and any3 / any2 run the shared-table
+kernel."""
 import numpy as np
 import pytest
 import torch

@@ -561,7 +561,8 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   // of the chunk) and this lane's alpha/beta pairs of the chunk's group.
   const uint8_t* abase = p.packed + p.ab_off + 16 * g;
   uint4 xn[NX][2], scn;
-  int last_grp = -1;
+  int last_grp = -1, pf_grp = -1;
+  const int pf_lim = ((p.n + 31) >> 5) * p.groups;   // scale records in the packed weight
   ChunkCursor<NW> xc;   // the chunk whose operands load next
   xc.start(P0, P1, u_lo, u_hi, kc, warp);
   auto next_operands = [&]() {
@@ -576,6 +577,10 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
     const int grp = xc.panel * p.groups + ((c * kChunkCols) >> p.g_shift);
     if (!kRowPair) {
       scn = ld_nc_v4(abase + ((size_t)grp << 7));
+      if (grp != pf_grp && grp + 1 < pf_lim) {   // the next group's record into L2 (measured: down
+        pf_grp = grp;                            // 4096 x 14336 at M = 16, 17.0 -> 15.5 us)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(abase + ((size_t)(grp + 1) << 7)));
+      }
     } else if (grp != last_grp) {   // a new group: its alpha/beta (read once, not kept in L1)
       scn = ld_stream_v4(abase + ((size_t)grp << 7));
       last_grp = grp;

@@ -133,6 +133,25 @@ def test_linear_edge_shapes(n, k, g, m):
     check_linear(y, x, q)
 
 
+@pytest.mark.parametrize("n,k,m", [(4096, 4096, 16), (4096, 4096, 2), (1024, 4096, 12), (1024, 4096, 3)])
+def test_linear_x_on_16_byte_boundary(n, k, m):
+    # x that starts 16 bytes past a 32-byte boundary takes the 128-bit
+    # activation loads instead of the 256-bit ones: same result bit for bit
+    q, s = quantized(n, k, 128, layer=f"xal{n}x{k}", iters=4)
+    xb = synth.activations_bf16(m, s, 70 + m, layer=f"xal{n}x{k}")
+    packed = pack_dev(q)
+    buf = torch.zeros(m * k + 16, dtype=torch.int16, device="cuda:0")
+    assert buf.data_ptr() % 32 == 0
+    x_off = buf[8:8 + m * k].view(m, k)
+    x_off.copy_(to_dev(xb).view(m, k))
+    assert x_off.data_ptr() % 32 == 16
+    y_off = a4.any4_linear(x_off.view(torch.bfloat16), packed, n, k, 128)
+    y_al = a4.any4_linear(bf16_dev(xb), packed, n, k, 128)
+    torch.cuda.synchronize()
+    assert torch.equal(y_off.view(torch.int16), y_al.view(torch.int16))
+    check_linear(y_off, xb, q)
+
+
 def test_linear_repeatable_and_workspace_restored():
     q, s = quantized(1024, 4096, 128, layer="rep", iters=4)
     x = bf16_dev(synth.activations_bf16(16, s, 6, layer="rep"))

@@ -95,13 +95,26 @@ def _dev(t: torch.Tensor, name: str, itemsize: int, shape=None) -> int:
         raise ValueError(f"{name} must have {itemsize}-byte elements, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != shape:
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     return t.data_ptr()
 
 
+# The current stream's raw handle without building a torch Stream object (the
+# binding's per-call cost bounds back-to-back calls of small shapes).
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(device.index if device.index is not None else torch.cuda.current_device())
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def _stream_of(t: torch.Tensor) -> int:
+    if _raw_stream is not None:
+        return _raw_stream(t.get_device())
+    return torch.cuda.current_stream(t.device).cuda_stream
 
 
 def any4_packed_bytes(n: int, k: int, group: int) -> int:
@@ -220,9 +233,11 @@ def any4_linear(x: torch.Tensor, packed: torch.Tensor, n: int, k: int, group: in
         out = torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
     if workspace is None:
         workspace = workspace_for(m, n, k, group, x.device)
-    _check(lib.any4_linear(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
-                           _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
-                           workspace.numel(), _stream(x.device)))
+    st = lib.any4_linear(_dev(x, "x", 2, (m, k)), _dev(packed, "packed", 1), m, n, k, group,
+                         _dev(out, "out", 2, (m, n)), _dev(workspace, "workspace", 1),
+                         workspace.numel(), _stream_of(x))
+    if st != ANY4_OK:
+        raise Any4Error(st)
     return out
 
 

@@ -66,18 +66,44 @@ def mixed(n: int, k: int, g: int, rows: tuple, seed: int = 0, layer: str = "w",
     return oracle.Any4Tensors(idx, lut, a, b, g), s
 
 
-def sample_rows(n: int, count: int = 48, seed: int = 0, whole_panels: int = 4) -> tuple:
+def split_panels(n: int, k: int, g: int, m: int = 1, bits: int = 4) -> list:
+    """32-row panels whose K range the any4_linear launch for this shape splits
+    between thread blocks (stream-K): a block owns units (panel, 64-column
+    chunk) floor(b*U/C) .. floor((b+1)*U/C) - 1 of U = panels * K/64, so a
+    block boundary that falls inside a panel splits it (that panel is the
+    last of block b - 1 and the first of block b). Empty when the launch
+    gives whole panels or clusters to blocks."""
+    import learned_bit_lut_b200 as a4
+    blocks, cluster = a4.any4_linear_grid(m, n, k, g, bits=bits)
+    panels, kc = (n + 31) // 32, k // 64
+    units = panels * kc
+    if cluster > 1 or blocks * kc == units:
+        return []
+    cuts = (b * units // blocks for b in range(1, blocks))
+    return sorted({u // kc for u in cuts if u % kc})
+
+
+def sample_rows(n: int, count: int = 48, seed: int = 0, whole_panels: int = 4, split_of=None) -> tuple:
     """Rows of the first and last tiles, spread random rows, and every row of
     ``whole_panels`` 32-row panels (the first, the last and random ones).
 
     At the benchmark shapes every panel of the any4 decode kernel is split
     along K between several warps and finished by the last one to arrive, so
-    whole panels check that reduction element by element."""
+    whole panels check that reduction element by element. With ``split_of =
+    (k, g)`` the random panels are drawn from the panels that the launch
+    splits between thread blocks (``split_panels``; the first and the last
+    of them always), which checks the stream-K finisher element by element."""
     g = np.random.default_rng(seed)
     pick = set(range(min(16, n))) | set(range(max(0, n - 16), n))
     pick |= set(g.choice(n, size=min(n, count), replace=False).tolist())
     panels = (n + 31) // 32
-    chosen = {0, panels - 1} | set(g.choice(panels, size=min(panels, max(0, whole_panels - 2)), replace=False).tolist())
+    chosen = {0, panels - 1}
+    pool = split_panels(n, *split_of) if split_of is not None else []
+    if pool:
+        chosen |= {pool[0], pool[-1]}
+        chosen |= set(g.choice(pool, size=min(len(pool), max(0, whole_panels - 2)), replace=False).tolist())
+    else:
+        chosen |= set(g.choice(panels, size=min(panels, max(0, whole_panels - 2)), replace=False).tolist())
     for p in sorted(chosen):
         pick |= set(range(32 * p, min(n, 32 * p + 32)))
     return tuple(sorted(pick))

@@ -51,7 +51,7 @@ def test_bits_dequant_bitexact_and_linear(bits, n, k, g):
 @pytest.mark.parametrize("m", [1, 16])
 def test_bits_llama3_8b_gate_sampled(bits, m):
     n, k, g = 14336, 4096, 128
-    rows = sample_rows(n, 32, seed=bits)
+    rows = sample_rows(n, 32, seed=bits, split_of=(k, g, 1, bits))
     idx, lut, al, be = synth.random_any4(n, k, g, 0, layer=f"bgate{bits}")
     mask = np.uint8((1 << bits) - 1)
     idx = (idx & mask) | (idx & np.uint8(mask << 4))   # both nibbles below 2^bits

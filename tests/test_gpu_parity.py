@@ -14,7 +14,7 @@ import learned_bit_lut_b200 as a4
 import oracle
 import synth
 from gpu_util import (bf16_dev, bits_host, check_linear, mixed, pack_dev, quantized,
-                      require_gpu, sample_rows, to_dev)
+                      require_gpu, sample_rows, split_panels, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -105,7 +105,9 @@ def test_linear_4096(m):
 @pytest.mark.parametrize("m", [1, 2, 4, 8, 16])
 def test_linear_llama3_8b_mlp(shape, m):
     n, k = shape
-    rows = sample_rows(n, 48, seed=n)
+    rows = sample_rows(n, 48, seed=n, split_of=(k, 128))
+    if n == 14336:   # 448 panels over the SMs: stream-K splits panels between blocks
+        assert set(split_panels(n, k, 128)) & {r // 32 for r in rows}
     q, s = mixed(n, k, 128, rows, layer=f"mlp{n}x{k}")
     x = synth.activations_bf16(m, s, 3, layer=f"mlp{n}x{k}")
     y = a4.any4_linear(bf16_dev(x), pack_dev(q), n, k, 128)
@@ -116,7 +118,7 @@ def test_linear_llama3_8b_mlp(shape, m):
 @pytest.mark.parametrize("m", [1, 16])
 def test_linear_llama3_70b_group_sweep(g, m):
     n, k = 28672, 8192
-    rows = sample_rows(n, 32, seed=g)
+    rows = sample_rows(n, 32, seed=g, split_of=(k, g))
     q, s = mixed(n, k, g, rows, layer=f"g{g}", kind="student_t", sigma=0.7)
     x = synth.activations_bf16(m, s, 4, layer=f"g{g}")
     y = a4.any4_linear(bf16_dev(x), pack_dev(q), n, k, g)
@@ -133,7 +135,7 @@ def test_linear_edge_shapes(n, k, g, m):
     check_linear(y, x, q)
 
 
-@pytest.mark.parametrize("n,k,m", [(4096, 4096, 16), (4096, 4096, 2), (1024, 4096, 12), (1024, 4096, 3)])
+@pytest.mark.parametrize("n,k,m", [(4096, 4096, 16), (4096, 4096, 7), (4096, 4096, 2), (1024, 4096, 12), (1024, 4096, 3)])
 def test_linear_x_on_16_byte_boundary(n, k, m):
     # x that starts 16 bytes past a 32-byte boundary takes the 128-bit
     # activation loads instead of the 256-bit ones: same result bit for bit

@@ -47,6 +47,14 @@ __device__ __forceinline__ void ld_nc_v8(const void* p, uint4& a, uint4& b) {
                : "l"(p));
 }
 
+// 256-bit load of read-only data kept in L1 ahead of other lines (evict_last);
+// the address must be 32-byte aligned.
+__device__ __forceinline__ void ld_keep_v8(const void* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.L1::evict_last.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+
 // 128-bit load of read-only data kept in L1 ahead of other lines (evict_last).
 __device__ __forceinline__ uint4 ld_keep_v4(const void* p) {
   uint4 v;

@@ -117,7 +117,7 @@ struct Params {
   int kc, groups, g_shift;                  // chunks per panel, groups per row, log2(G)
   int ctas;
   int cluster;                              // thread blocks per panel (a cluster), or 1
-  int x_vec32;                              // x is 32-byte aligned (M > 8: 256-bit activation loads)
+  int x_vec32;                              // x is 32-byte aligned (M > 4: 256-bit activation loads)
   long long units;
   size_t w_off, lut_off, ab_off;
 };
@@ -572,7 +572,9 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
 #pragma unroll
     for (int h = 0; h < NX; ++h) {
       const uint16_t* src = xrow[h] + (size_t)c * kChunkCols;
-      if (kRowPair) {
+      if (XV8 && kRowPair) {   // one 32-byte request per lane (M <= 8: kept in L1)
+        ld_keep_v8(src, xn[h][0], xn[h][1]);
+      } else if (kRowPair) {
         xn[h][0] = ld_keep_v4(src);
         xn[h][1] = ld_keep_v4(src + 8);
       } else if (XV8) {   // one 32-byte request per lane (measured: gate/up 18.9 -> 17.9 us)
@@ -748,8 +750,8 @@ template <int MODE, int BITS>
 cudaError_t allow_smem_mode() {
   cudaError_t e = cudaFuncSetAttribute(linear_kernel<MODE, BITS, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<MODE>::kSmemBytes);
-  if (e == cudaSuccess && MODE == 2)
-    e = cudaFuncSetAttribute(linear_kernel<MODE, BITS, MODE == 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (e == cudaSuccess && MODE >= 1)
+    e = cudaFuncSetAttribute(linear_kernel<MODE, BITS, MODE >= 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<MODE>::kSmemBytes);
   return e;
 }
@@ -794,7 +796,9 @@ cudaError_t launch_mode(const Params& p, const LinearPlan& plan, cudaStream_t st
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = plan.cluster > 1 ? 2 : 1;
-  if (MODE == 2 && p.x_vec32) return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS, MODE == 2>, p);
+  // 256-bit activation loads: measured faster at M = 5..16 (M = 8 down
+  // 4096 x 14336: 14.3 -> 13.9 us), no gain at M <= 4
+  if (MODE >= 1 && p.x_vec32) return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS, MODE >= 1>, p);
   return cudaLaunchKernelEx(&cfg, linear_kernel<MODE, BITS, false>, p);
 }
 

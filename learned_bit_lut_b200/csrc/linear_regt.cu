@@ -202,7 +202,10 @@ __global__ void __launch_bounds__(RegtCfg<NT8>::kThreads, 1) linear_regt_kernel(
     return;
   }
   if (receiver) {
-    // every other rank sends; rank 0 may not exit before their bytes land
+    // every other rank sends; rank 0 may not exit before their bytes land.
+    // The other ranks wait on nothing before they send (their loads and
+    // decode only), so the bound is a safety net that a running cluster
+    // never reaches: the cluster's blocks are co-scheduled.
     bool ok = mbar_try_wait(recv_bar, 0u);
     if (!ok) {
       const long long t0 = clock64();

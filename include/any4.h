@@ -126,6 +126,27 @@ ANY4_API size_t any4_linear_workspace_bytes(int m, int n, int k, int group);
  */
 ANY4_API int any4_linear_grid(int bits, int m, int n, int k, int group, int* blocks, int* cluster);
 
+/* Kernels of any4_linear / any4_linear_bits (any4_linear_kernel). */
+typedef enum {
+    ANY4_KERNEL_SHARED_TABLES = 1,    /* M <= 16: row-pair tables in shared memory (the general decode) */
+    ANY4_KERNEL_REGISTER_TABLES = 2,  /* M <= 16, any4, a short K split per cluster block: row tables in
+                                         registers, byte-permute decode */
+    ANY4_KERNEL_PREFILL_FUSED = 3,    /* 16 < M <= 512, any4: decode into the tcgen05 GEMM's shared memory */
+    ANY4_KERNEL_PREFILL_GEMM = 4      /* other M > 16: dequantize into the workspace, then the GEMM */
+} any4_kernel;
+
+/*
+ * any4_linear_kernel - which kernel any4_linear / any4_linear_bits run for
+ * this shape on the current device (introspection; no launch). The explainer
+ * (10100.com article 149119421, section 3) keeps each row's table next to the
+ * arithmetic; which form of it a shape gets is a launch decision of this
+ * library, fixed by the shape and the device's SM count.
+ *
+ * Returns an any4_kernel value (> 0), ANY4_ESHAPE for a shape or bit width
+ * the calls reject, or ANY4_ECUDA if the device cannot be queried.
+ */
+ANY4_API int any4_linear_kernel(int bits, int m, int n, int k, int group);
+
 /*
  * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
  *

@@ -10,7 +10,7 @@ streams.
 from ._lib import (ANY4_EALIGN, ANY4_ECUDA, ANY4_EINVAL, ANY4_ESHAPE, ANY4_EWORKSPACE,
                    ANY4_FORMAT_FP4, ANY4_FORMAT_INT4, ANY4_FORMAT_NF4, ANY4_OK, EXPORTED, FORMATS,
                    LIB_PATH, Any4Error, any4_dequant, any4_format_lut, any4_linear,
-                   any4_linear_grid, any4_linear_noalloc, any4_linear_workspace_bytes, noalloc_status, any4_pack,
+                   any4_linear_grid, any4_linear_kernel, KERNELS, any4_linear_noalloc, any4_linear_workspace_bytes, noalloc_status, any4_pack,
                    any4_pack_format,
                    any4_packed_bytes, any4_quantize, any4_strerror, lib, workspace_for,
                    any4_packed_bytes_bits, any4_pack_bits, any4_dequant_bits, any4_linear_bits)
@@ -18,6 +18,6 @@ from ._lib import (ANY4_EALIGN, ANY4_ECUDA, ANY4_EINVAL, ANY4_ESHAPE, ANY4_EWORK
 __all__ = ["any4_quantize", "any4_pack", "any4_pack_bits", "any4_dequant_bits", "any4_linear_bits",
            "any4_packed_bytes_bits", "any4_pack_format", "any4_format_lut", "FORMATS", "ANY4_FORMAT_INT4",
            "ANY4_FORMAT_NF4", "ANY4_FORMAT_FP4", "any4_dequant", "any4_linear", "any4_linear_noalloc", "noalloc_status", "any4_packed_bytes",
-           "any4_linear_workspace_bytes", "any4_linear_grid", "any4_strerror", "Any4Error", "workspace_for", "lib",
+           "any4_linear_workspace_bytes", "any4_linear_grid", "any4_linear_kernel", "KERNELS", "any4_strerror", "Any4Error", "workspace_for", "lib",
            "LIB_PATH", "EXPORTED", "ANY4_OK", "ANY4_EINVAL", "ANY4_EALIGN", "ANY4_ESHAPE",
            "ANY4_EWORKSPACE", "ANY4_ECUDA"]

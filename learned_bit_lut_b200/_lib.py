@@ -37,6 +37,8 @@ lib.any4_linear_workspace_bytes_bits.argtypes = [_c_int, _c_int, _c_int, _c_int,
 lib.any4_linear_workspace_bytes_bits.restype = _c_size
 lib.any4_linear_grid.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int, _p, _p]
 lib.any4_linear_grid.restype = _c_int
+lib.any4_linear_kernel.argtypes = [_c_int, _c_int, _c_int, _c_int, _c_int]
+lib.any4_linear_kernel.restype = _c_int
 lib.any4_linear.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p, _c_size, _p]
 lib.any4_linear.restype = _c_int
 lib.any4_linear_noalloc.argtypes = [_p, _p, _c_int, _c_int, _c_int, _c_int, _p, _p]
@@ -63,7 +65,7 @@ lib.any4_last_cuda_error.argtypes = []
 lib.any4_last_cuda_error.restype = _c_int
 
 EXPORTED = ("any4_packed_bytes", "any4_pack", "any4_dequant", "any4_linear_workspace_bytes",
-            "any4_linear_workspace_bytes_bits", "any4_linear_grid",
+            "any4_linear_workspace_bytes_bits", "any4_linear_grid", "any4_linear_kernel",
             "any4_linear", "any4_linear_noalloc", "any4_noalloc_status_word", "any4_quantize", "any4_format_lut",
             "any4_pack_format", "any4_packed_bytes_bits", "any4_pack_bits", "any4_dequant_bits",
             "any4_linear_bits", "any4_strerror", "any4_last_cuda_error")
@@ -123,6 +125,17 @@ def any4_packed_bytes(n: int, k: int, group: int) -> int:
 
 def any4_linear_workspace_bytes(m: int, n: int, k: int, group: int) -> int:
     return lib.any4_linear_workspace_bytes(m, n, k, group)
+
+
+KERNELS = {1: "shared_tables", 2: "register_tables", 3: "prefill_fused", 4: "prefill_gemm"}
+
+
+def any4_linear_kernel(m: int, n: int, k: int, group: int, bits: int = 4) -> str:
+    """Name of the kernel any4_linear runs for this shape on the current device."""
+    code = lib.any4_linear_kernel(bits, m, n, k, group)
+    if code < 0:
+        raise Any4Error(code)
+    return KERNELS[code]
 
 
 def any4_linear_grid(m: int, n: int, k: int, group: int, bits: int = 4) -> tuple[int, int]:

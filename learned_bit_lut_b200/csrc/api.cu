@@ -119,6 +119,18 @@ int any4_linear_grid(int bits, int m, int n, int k, int group, int* blocks, int*
   return ANY4_OK;
 }
 
+int any4_linear_kernel(int bits, int m, int n, int k, int group) {
+  if (!any4::bits_ok(bits) || m < 1 || m > any4::kMaxTokens || !any4::shape_ok(n, k, group))
+    return ANY4_ESHAPE;
+  int sms = 0;
+  const int st = current_sm_count(&sms);
+  if (st != ANY4_OK) return st;
+  const any4::Layout L = any4::make_layout(n, k, group, bits);
+  const any4::LinearPlan plan = any4::plan_linear(m, L, sms);
+  if (plan.mode == 3) return any4::prefill_fused(L, m) ? ANY4_KERNEL_PREFILL_FUSED : ANY4_KERNEL_PREFILL_GEMM;
+  return plan.regt ? ANY4_KERNEL_REGISTER_TABLES : ANY4_KERNEL_SHARED_TABLES;
+}
+
 int any4_linear(const uint16_t* x, const void* packed, int m, int n, int k, int group,
                 uint16_t* y, void* workspace, size_t workspace_bytes, any4_stream_t stream) {
   if (!x || !packed || !y || !workspace) return ANY4_EINVAL;

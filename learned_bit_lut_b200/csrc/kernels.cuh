@@ -50,6 +50,7 @@ constexpr unsigned kStatusWaitTimeout = 1u;
 // M > 16 (prefill): bf16 W_hat scratch at prefill_scratch_offset() of the
 // workspace, then a tcgen05 GEMM (prefill.cu).
 size_t prefill_scratch_offset();
+bool prefill_fused(const Layout& L, int m);   // M > 16 decodes into the GEMM's shared memory
 size_t prefill_workspace_bytes(const Layout& L, int m, int num_sms);
 cudaError_t launch_prefill(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
                            void* workspace, int num_sms, cudaStream_t stream);

@@ -792,6 +792,8 @@ cudaError_t launch_fused(const uint16_t* x, const uint8_t* packed, const Layout&
 
 size_t prefill_scratch_offset() { return kHeaderBytes; }
 
+bool prefill_fused(const Layout& L, int m) { return fused_path(L, m); }
+
 int prefill_splits(const Layout& L, int m, int num_sms) {
   const int tiles = ((L.n + kBM - 1) / kBM) * ((m + kBN - 1) / kBN);
   const int kch = L.k / kBK;

@@ -135,3 +135,10 @@ def test_linear_grid_rejects_on_host():
     assert a4.lib.any4_linear_grid(5, 1, 4096, 4096, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE
     assert a4.lib.any4_linear_grid(4, 0, 4096, 4096, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE
     assert a4.lib.any4_linear_grid(4, 1, 4096, 4000, 128, ctypes.byref(b), ctypes.byref(c)) == a4.ANY4_ESHAPE
+
+
+def test_linear_kernel_rejects_on_host():
+    assert a4.lib.any4_linear_kernel(5, 1, 4096, 4096, 128) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_kernel(4, 0, 4096, 4096, 128) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_kernel(4, 1, 4096, 4000, 128) == a4.ANY4_ESHAPE
+    assert a4.lib.any4_linear_kernel(4, 1, 4095, 4096, 128) == a4.ANY4_ESHAPE

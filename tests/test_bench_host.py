@@ -73,6 +73,14 @@ def test_result_line_weak_scaling_and_roofline():
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "vs_baseline",
                 "dtype", "data", "config", "roofline", "gpu_launches", "clocks", "e2e", "cpu_baseline"):
         assert key in one
+    # the dominant kernel timed on its own sets the roofline, not the step
+    dom = {"bytes": 6_000_000_000, "ms": 3.0, "launches": 320}
+    three = bench.result_line(1, 200, 5, ms, step_bytes, n_calls, {}, 6457.4, "measured", {}, None, None, dom)
+    assert three["value"] == pytest.approx(one["value"])
+    assert three["roofline"]["achieved"] == pytest.approx(6_000_000_000 / 3.0e6)
+    assert three["roofline"]["launches_per_step"] == 320
+    if three["roofline"]["traffic"] is not None:
+        assert three["roofline"]["traffic"] == pytest.approx(bench.DRAM_PER_ALGO_BYTE * 6_000_000_000 / 320)
 
 
 def test_step_bytes_match_the_workload_table():

@@ -47,6 +47,10 @@ def test_cluster_grid(n, k, g, cl):
         assert cluster == cl and blocks == panels * cl
     blocks, cluster = a4.any4_linear_grid(17, n, k, g)   # prefill: no clusters
     assert cluster == 1
+    # which decode kernel splits the panels (any4 with at most 16 chunks per
+    # block: the register-table kernel)
+    want = "register_tables" if cl <= 4 and k // 64 <= 16 * cl else "shared_tables"
+    assert a4.any4_linear_kernel(1, n, k, g) == want
 
 
 @pytest.mark.parametrize("n,k,g,cl", SHAPES)

@@ -89,6 +89,16 @@ def test_prefill_repeatable_and_guard_rows_untouched():
     assert torch.all(buf[0] == 7) and torch.all(buf[m + 1] == 7)
 
 
+def test_prefill_kernel_choice():
+    # any4 up to 512 tokens decodes into the GEMM's shared memory; beyond that,
+    # and for any3 / any2, the weight is dequantized into the workspace first
+    assert a4.any4_linear_kernel(17, 4096, 4096, 128) == "prefill_fused"
+    assert a4.any4_linear_kernel(512, 4096, 4096, 128) == "prefill_fused"
+    assert a4.any4_linear_kernel(513, 4096, 4096, 128) == "prefill_gemm"
+    assert a4.any4_linear_kernel(40, 4096, 4096, 128, bits=3) == "prefill_gemm"
+    assert a4.any4_linear_kernel(16, 4096, 4096, 128) == "shared_tables"
+
+
 def test_prefill_workspace_size():
     n, k, g = 4096, 4096, 128
     header = STATUS_OFFSET + 256

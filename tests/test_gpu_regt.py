@@ -55,8 +55,12 @@ def test_regt_plan(n, k, g, c8, c16):
         blocks, cluster = a4.any4_linear_grid(m, n, k, g)
         if cl is not None:
             assert (blocks, cluster) == (panels * cl, cl)
+            assert a4.any4_linear_kernel(m, n, k, g) == "register_tables"
+        else:
+            assert a4.any4_linear_kernel(m, n, k, g) == "shared_tables"
     # the shared-table kernel keeps 3- and 2-bit weights
     assert a4.any4_linear_grid(1, 1024, 4096, 128, bits=3)[1] == 4
+    assert a4.any4_linear_kernel(1, 1024, 4096, 128, bits=3) == "shared_tables"
 
 
 @pytest.mark.parametrize("n,k,g,c8,c16", SHAPES)

@@ -132,7 +132,9 @@ typedef enum {
     ANY4_KERNEL_REGISTER_TABLES = 2,  /* M <= 16, any4, a short K split per cluster block: row tables in
                                          registers, byte-permute decode */
     ANY4_KERNEL_PREFILL_FUSED = 3,    /* 16 < M <= 512, any4: decode into the tcgen05 GEMM's shared memory */
-    ANY4_KERNEL_PREFILL_GEMM = 4      /* other M > 16: dequantize into the workspace, then the GEMM */
+    ANY4_KERNEL_PREFILL_GEMM = 4,     /* other M > 16: dequantize into the workspace, then the GEMM */
+    ANY4_KERNEL_SHARED_TABLES_DIRECT = 5  /* M <= 4, any4, few chunks per block: the shared row-pair tables
+                                             with each warp loading its own operands */
 } any4_kernel;
 
 /*

@@ -127,7 +127,8 @@ def any4_linear_workspace_bytes(m: int, n: int, k: int, group: int) -> int:
     return lib.any4_linear_workspace_bytes(m, n, k, group)
 
 
-KERNELS = {1: "shared_tables", 2: "register_tables", 3: "prefill_fused", 4: "prefill_gemm"}
+KERNELS = {1: "shared_tables", 2: "register_tables", 3: "prefill_fused", 4: "prefill_gemm",
+           5: "shared_tables_direct"}
 
 
 def any4_linear_kernel(m: int, n: int, k: int, group: int, bits: int = 4) -> str:

@@ -128,6 +128,7 @@ int any4_linear_kernel(int bits, int m, int n, int k, int group) {
   const any4::Layout L = any4::make_layout(n, k, group, bits);
   const any4::LinearPlan plan = any4::plan_linear(m, L, sms);
   if (plan.mode == 3) return any4::prefill_fused(L, m) ? ANY4_KERNEL_PREFILL_FUSED : ANY4_KERNEL_PREFILL_GEMM;
+  if (plan.small) return ANY4_KERNEL_SHARED_TABLES_DIRECT;
   return plan.regt ? ANY4_KERNEL_REGISTER_TABLES : ANY4_KERNEL_SHARED_TABLES;
 }
 

@@ -63,6 +63,7 @@ struct LinearPlan {
   int ctas;             // persistent thread blocks (one per SM at most)
   int cluster;          // thread blocks sharing one panel as a cluster (K slices), or 1
   bool regt;            // register-table kernel (linear_regt.cu) instead of linear.cu's
+  bool small;           // shared-table kernel without streaming structure (linear_small.cu)
   size_t partials_bytes;
   size_t workspace_bytes;
 };
@@ -75,6 +76,13 @@ int regt_warps(int m);
 int regt_max_cluster();
 cudaError_t launch_linear_regt(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
                                void* workspace, int cluster, cudaStream_t stream);
+
+// M <= 16, any4, few chunks per thread block: the row-pair tables in shared
+// memory, one cluster of `cluster` blocks per panel (linear_small.cu).
+int small_warps(int m);
+int small_max_cluster();
+cudaError_t launch_linear_small(const uint16_t* x, const uint8_t* packed, const Layout& L, int m, uint16_t* y,
+                                void* workspace, int cluster, cudaStream_t stream);
 
 cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout& L, int m,
                           uint16_t* y, void* workspace, const LinearPlan& plan,

@@ -82,6 +82,8 @@ constexpr int kConsumerBar = 1;              // named barrier of the consumer wa
 constexpr int kMaxCluster = 8;               // thread blocks sharing one panel (portable cluster size)
 constexpr int kMinClusterChunks = 16;        // chunks a block of such a cluster works on, at least
 constexpr int kRegtMaxChunks = 16;           // chunks per block up to which linear_regt.cu decodes
+constexpr int kSmallMaxTokens = 4;           // M up to which linear_small.cu takes the short splits
+constexpr int kSmallWholeMaxChunks = 64;     // ... and whole panels of at most this many chunks
 
 // MODE 0: M <= 4, MODE 1: M <= 8 (row-pair operands, one or two column tiles
 // of 4 tokens); MODE 2: M <= 16 (row operands, two 8-token column tiles).
@@ -899,22 +901,32 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   if (c < 1) c = 1;
   pl.ctas = (int)c;
   // a short K split over a cluster per panel (at most kRegtMaxChunks chunks
-  // per block, at least one per warp): the fixed cost of a panel's shared
-  // tables and barriers outweighs the decode, so the register-table kernel
-  // takes it, on its own cluster split (measured on B200: faster on such
-  // shapes, slower without a cluster or with idle warps)
+  // per block, at least one per warp): the fixed cost of this kernel's
+  // streaming structure outweighs the decode, so for M = 5..16 the
+  // register-table kernel takes it, on its own cluster split (measured on
+  // B200: faster on such shapes, slower without a cluster or with idle warps).
+  // For M <= 4 the same splits, and whole panels of up to
+  // kSmallWholeMaxChunks chunks, run the shared tables without the streaming
+  // structure (linear_small.cu; measured on B200: k/v 3.70 -> 3.25 us, q/o
+  // 4.64 -> 4.33 us at M = 1, slower than these kernels for M > 4).
   if (L.bits == 4 && L.panels <= num_sms) {
+    const bool direct = m <= kSmallMaxTokens;
+    const int warps = direct ? small_warps(m) : regt_warps(m);
     int s = 0;
     for (int q = regt_max_cluster(); q >= 2; q /= 2) {
-      if ((long long)L.panels * q <= num_sms && L.kchunks >= q * regt_warps(m)) {
+      if ((long long)L.panels * q <= num_sms && L.kchunks >= q * warps) {
         s = q;
         break;
       }
     }
     if (s > 0 && L.kchunks <= s * kRegtMaxChunks) {
-      pl.regt = true;
+      (direct ? pl.small : pl.regt) = true;
       pl.cluster = s;
       pl.ctas = L.panels * s;
+    } else if (direct && L.kchunks <= kSmallWholeMaxChunks) {
+      pl.small = true;
+      pl.cluster = 1;
+      pl.ctas = L.panels;
     }
   }
   // partial sums are only used without clusters, by at most one block per
@@ -931,6 +943,7 @@ cudaError_t launch_linear(const uint16_t* x, const uint8_t* packed, const Layout
                           cudaStream_t stream) {
   if (plan.mode == 3) return launch_prefill(x, packed, L, m, y, workspace, plan.ctas, stream);
   if (plan.regt) return launch_linear_regt(x, packed, L, m, y, workspace, plan.cluster, stream);
+  if (plan.small) return launch_linear_small(x, packed, L, m, y, workspace, plan.cluster, stream);
   cudaError_t e = allow_large_smem();
   if (e != cudaSuccess) return e;
   Params p{};

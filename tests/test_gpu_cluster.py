@@ -6,9 +6,9 @@ launch really is clustered, the linear layer's acceptance bar against the
 oracle for every decode mode (M = 1, 3, 8, 16), ragged K slices and a ragged
 last panel, any3 / any2, and that repeated calls are bit-identical. For any4
 the shapes with at most 16 chunks per block (1024 x 4096, 1008 x 4096 and
-2048 x 2048) take the register-table kernel, which splits the same
-way (tests/test_gpu_regt.py); the others and any3 / any2 run the shared-table
-kernel."""
+2048 x 2048) take the short-split kernels, which split the same way
+(tests/test_gpu_regt.py); the others and any3 / any2 run the streaming
+shared-table kernel."""
 import numpy as np
 import pytest
 import torch
@@ -48,9 +48,10 @@ def test_cluster_grid(n, k, g, cl):
     blocks, cluster = a4.any4_linear_grid(17, n, k, g)   # prefill: no clusters
     assert cluster == 1
     # which decode kernel splits the panels (any4 with at most 16 chunks per
-    # block: the register-table kernel)
-    want = "register_tables" if cl <= 4 and k // 64 <= 16 * cl else "shared_tables"
-    assert a4.any4_linear_kernel(1, n, k, g) == want
+    # block: the short-split kernels)
+    short = cl <= 4 and k // 64 <= 16 * cl
+    assert a4.any4_linear_kernel(1, n, k, g) == ("shared_tables_direct" if short else "shared_tables")
+    assert a4.any4_linear_kernel(16, n, k, g) == ("register_tables" if short else "shared_tables")
 
 
 @pytest.mark.parametrize("n,k,g,cl", SHAPES)

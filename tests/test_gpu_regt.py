@@ -1,10 +1,13 @@
-"""GPU parity of the register-table decode (any4, M <= 16, short K splits).
+"""GPU parity of the short-K-split decode kernels (any4, M <= 16).
 
 Shapes whose 32-row panels fit the SMs two or four times over, with at most
-16 chunks of 64 columns per thread block and at least one per warp, run the
-register-table kernel: every lane holds the 16-entry tables of its four rows
-as byte planes, decodes with byte permutes, and a cluster of 2 or 4 blocks
-per panel adds its K slices in rank order through distributed shared memory.
+16 chunks of 64 columns per thread block and at least one per warp, run on a
+cluster of 2 or 4 blocks per panel that adds its K slices in rank order
+through distributed shared memory: for M = 5..16 the register-table kernel
+(every lane holds the 16-entry tables of its four rows as byte planes and
+decodes with byte permutes), for M <= 4 the shared row-pair tables with each
+warp loading its own operands (which also takes whole panels of at most 64
+chunks at M <= 4).
 Checks the plan (grid and cluster size on a 148-SM B200), the linear layer's
 acceptance bar and the tight elementwise bar against the oracle for token
 counts of both operand tiles (1-8 and 9-16 tokens), ragged last panels
@@ -51,13 +54,16 @@ def test_regt_plan(n, k, g, c8, c16):
     if sm_count() != 148:
         pytest.skip("cluster sizes are stated for a 148-SM B200")
     panels = (n + 31) // 32
-    for m, cl in ((1, c8), (8, c8), (9, c16), (16, c16)):
+    for m, cl in ((1, c8), (4, c8), (5, c8), (8, c8), (9, c16), (16, c16)):
         blocks, cluster = a4.any4_linear_grid(m, n, k, g)
+        kernel = a4.any4_linear_kernel(m, n, k, g)
         if cl is not None:
             assert (blocks, cluster) == (panels * cl, cl)
-            assert a4.any4_linear_kernel(m, n, k, g) == "register_tables"
+            assert kernel == ("shared_tables_direct" if m <= 4 else "register_tables")
+        elif m <= 4 and k // 64 <= 64:   # whole panels, one block each
+            assert (blocks, cluster, kernel) == (panels, 1, "shared_tables_direct")
         else:
-            assert a4.any4_linear_kernel(m, n, k, g) == "shared_tables"
+            assert kernel == "shared_tables"
     # the shared-table kernel keeps 3- and 2-bit weights
     assert a4.any4_linear_grid(1, 1024, 4096, 128, bits=3)[1] == 4
     assert a4.any4_linear_kernel(1, 1024, 4096, 128, bits=3) == "shared_tables"

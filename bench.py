@@ -209,7 +209,8 @@ def result_line(world: int, steps: int, warmup: int, ms_step: float, step_bytes:
                      "launches_per_step": dominant["launches"],
                      "note": ("achieved = the kernel's algorithmic bytes per launch over its mean launch "
                               "time, from its own calls of the step replayed back to back; the k/v calls "
-                              "run linear_regt_kernel")},
+                              "and the M=1 q/o calls run linear_small_kernel (M=1) or "
+                              "linear_regt_kernel (M=16)")},
         "gpu_launches": n_calls * steps,
         "clocks": clocks,
         "e2e": e2e,

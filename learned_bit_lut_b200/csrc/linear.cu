@@ -83,7 +83,7 @@ constexpr int kMaxCluster = 8;               // thread blocks sharing one panel 
 constexpr int kMinClusterChunks = 16;        // chunks a block of such a cluster works on, at least
 constexpr int kRegtMaxChunks = 16;           // chunks per block up to which linear_regt.cu decodes
 constexpr int kSmallMaxTokens = 4;           // M up to which linear_small.cu takes the short splits
-constexpr int kSmallWholeMaxChunks = 64;     // ... and whole panels of at most this many chunks
+constexpr int kSmallWholeMaxChunks = 128;    // ... and whole panels of at most this many chunks
 
 // MODE 0: M <= 4, MODE 1: M <= 8 (row-pair operands, one or two column tiles
 // of 4 tokens); MODE 2: M <= 16 (row operands, two 8-token column tiles).
@@ -906,9 +906,11 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
   // register-table kernel takes it, on its own cluster split (measured on
   // B200: faster on such shapes, slower without a cluster or with idle warps).
   // For M <= 4 the same splits, and whole panels of up to
-  // kSmallWholeMaxChunks chunks, run the shared tables without the streaming
-  // structure (linear_small.cu; measured on B200: k/v 3.70 -> 3.25 us, q/o
-  // 4.64 -> 4.33 us at M = 1, slower than these kernels for M > 4).
+  // kSmallWholeMaxChunks chunks where this kernel would run whole panels
+  // too, run the shared tables without the streaming structure
+  // (linear_small.cu; measured on B200 at M = 1: k/v 3.70 -> 3.25 us, q/o
+  // 4.64 -> 4.33 us, 4096 x 8192 7.12 -> 6.70 us, 4096 x 14336 equal; slower
+  // than these kernels for M > 4).
   if (L.bits == 4 && L.panels <= num_sms) {
     const bool direct = m <= kSmallMaxTokens;
     const int warps = direct ? small_warps(m) : regt_warps(m);
@@ -923,7 +925,7 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
       (direct ? pl.small : pl.regt) = true;
       pl.cluster = s;
       pl.ctas = L.panels * s;
-    } else if (direct && L.kchunks <= kSmallWholeMaxChunks) {
+    } else if (direct && pl.cluster == 1 && L.kchunks <= kSmallWholeMaxChunks) {   // whole panels here too
       pl.small = true;
       pl.cluster = 1;
       pl.ctas = L.panels;

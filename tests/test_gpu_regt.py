@@ -6,8 +6,8 @@ cluster of 2 or 4 blocks per panel that adds its K slices in rank order
 through distributed shared memory: for M = 5..16 the register-table kernel
 (every lane holds the 16-entry tables of its four rows as byte planes and
 decodes with byte permutes), for M <= 4 the shared row-pair tables with each
-warp loading its own operands (which also takes whole panels of at most 64
-chunks at M <= 4).
+warp loading its own operands (which also takes whole panels of at most 128
+chunks at M <= 4 where the streaming kernel would run whole panels too).
 Checks the plan (grid and cluster size on a 148-SM B200), the linear layer's
 acceptance bar and the tight elementwise bar against the oracle for token
 counts of both operand tiles (1-8 and 9-16 tokens), ragged last panels
@@ -60,10 +60,8 @@ def test_regt_plan(n, k, g, c8, c16):
         if cl is not None:
             assert (blocks, cluster) == (panels * cl, cl)
             assert kernel == ("shared_tables_direct" if m <= 4 else "register_tables")
-        elif m <= 4 and k // 64 <= 64:   # whole panels, one block each
-            assert (blocks, cluster, kernel) == (panels, 1, "shared_tables_direct")
-        else:
-            assert kernel == "shared_tables"
+        else:   # these shapes split panels over a cluster of the streaming kernel
+            assert kernel == "shared_tables" and cluster > 1
     # the shared-table kernel keeps 3- and 2-bit weights
     assert a4.any4_linear_grid(1, 1024, 4096, 128, bits=3)[1] == 4
     assert a4.any4_linear_kernel(1, 1024, 4096, 128, bits=3) == "shared_tables"

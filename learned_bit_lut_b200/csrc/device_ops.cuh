@@ -177,9 +177,13 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, flo
       : "memory");
 }
 
-// Every thread of every block of the cluster.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+// Every thread of every block of the cluster, with a relaxed arrive: enough
+// to publish mbarrier initialisations that a fence.mbarrier_init.release
+// .cluster ordered before it (the other blocks then complete transactions on
+// them), without making all earlier memory operations visible cluster-wide
+// (measured on B200: 0.4-0.5 us less per call of a 4-block cluster).
+__device__ __forceinline__ void cluster_sync_init() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) {

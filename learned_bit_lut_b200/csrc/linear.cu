@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(Cfg<MODE>::kThreads, 1) linear_kernel(const Pa
   fence_mbar_init();
   if (tid == 0 && receiver) mbar_arrive_expect_tx(recv_bar, (uint32_t)((csz - 1) * 32 * NF * 4));
   __syncthreads();
-  if (csz > 1) cluster_sync_all();   // rank 0's receive barrier is armed before any rank sends
+  if (csz > 1) cluster_sync_init();   // rank 0's receive barrier is armed before any rank sends
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // =========================== producer warp ===============================

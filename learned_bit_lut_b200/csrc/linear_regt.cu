@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(RegtCfg<NT8>::kThreads, 1) linear_regt_kernel(
     mbar_arrive_expect_tx(recv_bar, (uint32_t)((csz - 1) * C::kTileBytes));
   }
   __syncthreads();
-  if (csz > 1) cluster_sync_all();   // rank 0's receive barrier is armed before any rank sends
+  if (csz > 1) cluster_sync_init();   // rank 0's receive barrier is armed before any rank sends
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // this warp's chunks: its share of the block's K slice of panel P

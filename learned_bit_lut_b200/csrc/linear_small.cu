@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(SmallCfg<MODE>::kThreads, 1) linear_small_kern
     }
   }
   __syncthreads();
-  if (csz > 1) cluster_sync_all();   // rank 0's receive barrier is armed before any rank sends
+  if (csz > 1) cluster_sync_init();   // rank 0's receive barrier is armed before any rank sends
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- activations and scales (after the grid-dependency wait)

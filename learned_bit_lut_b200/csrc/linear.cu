@@ -915,7 +915,7 @@ LinearPlan plan_linear(int m, const Layout& L, int num_sms) {
     const bool direct = m <= kSmallMaxTokens;
     const int warps = direct ? small_warps(m) : regt_warps(m);
     int s = 0;
-    for (int q = regt_max_cluster(); q >= 2; q /= 2) {
+    for (int q = direct ? small_max_cluster() : regt_max_cluster(); q >= 2; q /= 2) {   // each kernel's receive buffers
       if ((long long)L.panels * q <= num_sms && L.kchunks >= q * warps) {
         s = q;
         break;

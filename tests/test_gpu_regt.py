@@ -137,3 +137,19 @@ def test_regt_one_hot_columns_read_back_indices(m):
     idx[:, 1::2] = idx_nib >> 4
     expect = (idx[:, cols] - 8).T.astype(np.float32)
     assert np.array_equal(y, expect)
+
+
+@pytest.mark.parametrize("m", [1, 4])
+def test_direct_kernel_whole_panels_up_to_128_chunks(m):
+    # 128 panels of 128 chunks: at M <= 4 one block per panel of the shared
+    # tables with per-warp loads (each warp takes 8 chunks in turn)
+    from gpu_util import mixed, sample_rows
+    n, k, g = 4096, 8192, 128
+    if sm_count() >= 128:
+        assert a4.any4_linear_kernel(m, n, k, g) == "shared_tables_direct"
+        assert a4.any4_linear_grid(m, n, k, g) == (128, 1)
+    rows = sample_rows(n, 32, seed=m, whole_panels=4)
+    q, s = mixed(n, k, g, rows, layer="direct_long")
+    x = synth.activations_bf16(m, s, 80 + m, layer="direct_long")
+    y = a4.any4_linear(bf16_dev(x), pack_dev(q), n, k, g)
+    check_linear(y, x, q, rows)

@@ -31,7 +31,9 @@
 //    of (32-row panel, 64-column chunk) units: stream-K over all SMs when
 //    panels outnumber them, one whole panel per block when they do not, and
 //    a cluster of 2-8 blocks per panel (K slices) when whole panels would
-//    leave most SMs idle. For each panel its
+//    leave most SMs idle. (Where a block would get only a few chunks,
+//    plan_linear hands the shape to linear_small.cu or linear_regt.cu
+//    instead, which skip this kernel's streaming structure.) For each panel its
 //    consumer warps (16 for M <= 4, 12 for M <= 8, 8 for M <= 16: what the
 //    register file and shared memory hold) build the 16 row-pair tables
 //    (64 KB) once, then split the panel's chunks. A producer warp streams

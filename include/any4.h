@@ -153,7 +153,12 @@ ANY4_API int any4_linear_kernel(int bits, int m, int n, int k, int group);
  * any4_linear - y = x . W_hat^T, the any4 mixed-precision linear layer.
  *
  *   m          tokens, 1 .. 2^20. M <= 16 (decode, explainer section 3's
- *              batch 1-16) runs the fused dequant-and-contract kernel below.
+ *              batch 1-16) runs a fused dequant-and-contract kernel, as
+ *              below; which one (the streaming shared-table kernel, or for
+ *              shapes with few chunks per thread block the shared tables
+ *              with per-warp loads at M <= 4 or the register tables at
+ *              M = 5-16) depends on the shape and is reported by
+ *              any4_linear_kernel.
  *              M > 16 (prefill) runs a tensor-core GEMM (tcgen05, fp32
  *              accumulation in tensor memory): up to M = 512 its A tiles are
  *              decoded from the packed weight straight into shared memory
@@ -180,8 +185,9 @@ ANY4_API int any4_linear_kernel(int bits, int m, int n, int k, int group);
  * by the block that holds their first columns: it waits for the others' fp32
  * partials (through the workspace, or within a cluster through distributed
  * shared memory) and adds them in a fixed order, so the result is
- * deterministic.
- * Every wait in the kernel is bounded (~2 s); if one gives up, the kernel
+ * deterministic (every kernel adds in a fixed order; two calls of the same
+ * shape on the same device give the same bits).
+ * Every wait in the kernels is bounded (~2-4 s); if one gives up, the kernel
  * completes without hanging and the first 32-bit word of the workspace's
  * reserved area (byte offset 65536*4) is set non-zero. It is zero after
  * every normal call.

@@ -81,6 +81,10 @@ __global__ void __launch_bounds__(SmallCfg<MODE>::kThreads, 1) linear_small_kern
     return;
   }
 
+  // the next kernel on the stream may start launching (it waits for this
+  // grid before it touches what this one writes)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
   // ---- immutable inputs first: this thread's table-build entries, the
   // warp's first index words
   // 512 build tasks (pair slot, high nibble, low-nibble half), kPer per thread
@@ -136,7 +140,6 @@ __global__ void __launch_bounds__(SmallCfg<MODE>::kThreads, 1) linear_small_kern
   }
   __syncthreads();
   if (csz > 1) cluster_sync_init();   // rank 0's receive barrier is armed before any rank sends
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- activations and scales (after the grid-dependency wait)
   asm volatile("griddepcontrol.wait;" ::: "memory");

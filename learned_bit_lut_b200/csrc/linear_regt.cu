@@ -1,5 +1,5 @@
-// any4_linear, M <= 16, for shapes with few 32-row panels: row tables held in
-// registers instead of shared memory.
+// any4_linear, M = 5..16, for shapes with few 32-row panels: row tables held
+// in registers instead of shared memory.
 //
 // The explainer (10100.com, article 149119421, section 3) keeps each row's
 // table in registers and decodes with native instructions. On B200 that
@@ -9,7 +9,9 @@
 // (the Llama K/V projections, 1024 x 4096) a warp sees only one or two
 // chunks, and what a call then costs is its fixed work: building a 64 KB
 // row-pair table per block and the block barriers around it. This kernel has
-// none of it:
+// none of it (for M <= 4, where the contraction is lighter, the shared tables
+// with per-warp loads of linear_small.cu measured faster and take those
+// shapes):
 //
 //  * grid: s thread blocks per panel (a thread-block cluster, s = 1, 2, 4), each
 //    on a contiguous K slice; inside a block every warp takes its own chunks;
